@@ -1,0 +1,194 @@
+"""fp64 CPU oracle (ctypes wrapper around ``dit_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``, never by the CUDA library or its
+Python binding.  It shares no code with the CUDA path.
+
+Every function here follows the definitions cited in ``dit_oracle.c``:
+softmax attention (Z-Image FlashAttention-2 page, opening section; TMAP
+image-to-video page, FLOP table), the first-block-cache residual difference
+(ParaAttention page, "First Block Cache") and the 8-bit quantiser with its
+zero-scale guard (TMAP page, "optimising operator details").
+
+``emulated_q8_attention`` is parity unpinned beyond its inputs: it replays the
+quantised arithmetic in fp64 to separate quantisation error from kernel error
+and is never the judged reference (the judged reference for the 8-bit path is
+the exact fp64 attention on the unquantised inputs).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dit_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_i64 = ctypes.c_int64
+_p = ctypes.c_void_p
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc + OpenMP (no fast-math: IEEE fp64/fp32)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-fno-fast-math", "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        lib.oracle_attn_f64.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_double, _p, _i64]
+        lib.oracle_attn_bf16in.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_double, _p, _i64]
+        lib.oracle_fbc_rel_l1.argtypes = [_p, _p, _i64, ctypes.c_int, ctypes.c_double, _p, _p]
+        lib.oracle_channel_mean.argtypes = [_p, _i64, _i64, _i64, _p]
+        lib.oracle_quant_int8_blocks.argtypes = [_p, _i64, _i64, _i64, _i64, _p, _p, _p]
+        lib.oracle_quant_e4m3_channels.argtypes = [_p, _i64, _i64, _i64, _p, _p]
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = ctypes.c_float
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def attention(q, k, v, scale: float | None = None, rows=None) -> np.ndarray:
+    """O = softmax(scale * Q K^T) V in fp64.
+
+    q, k, v: [B, H, N, d] as float64 arrays, or uint16 arrays of bf16 bits
+    (widened exactly).  ``scale`` defaults to 1/sqrt(d) computed in fp32 and
+    widened, the value the CUDA path receives.  ``rows``: optional query-row
+    indices; the result is then [B, H, len(rows), d].
+    """
+    B, H, N, d = q.shape
+    assert k.shape == (B, H, N, d) and v.shape == (B, H, N, d)
+    if scale is None:
+        scale = float(np.float32(1.0) / np.sqrt(np.float32(d)))
+    nrows = N
+    rows_arr = None
+    if rows is not None:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        assert rows_arr.ndim == 1 and (rows_arr >= 0).all() and (rows_arr < N).all()
+        nrows = len(rows_arr)
+    out = np.empty((B, H, nrows, d), dtype=np.float64)
+    lib = _load()
+    rp = _ptr(rows_arr) if rows_arr is not None else None
+    if q.dtype == np.uint16:
+        q, k, v = (np.ascontiguousarray(t, dtype=np.uint16) for t in (q, k, v))
+        rc = lib.oracle_attn_bf16in(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d,
+                                    float(scale), rp, nrows)
+    else:
+        q, k, v = (np.ascontiguousarray(t, dtype=np.float64) for t in (q, k, v))
+        rc = lib.oracle_attn_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d,
+                                 float(scale), rp, nrows)
+    if rc != 0:
+        raise RuntimeError(f"oracle attention failed ({rc})")
+    return out
+
+
+def fbc_rel_l1(cur, prev, threshold: float):
+    """(rel, skip) for two residuals: fp32 arrays or uint16 bf16 bit arrays."""
+    cur = np.ascontiguousarray(cur).reshape(-1)
+    prev = np.ascontiguousarray(prev).reshape(-1)
+    assert cur.shape == prev.shape and cur.dtype == prev.dtype
+    if cur.dtype == np.float32:
+        dt = 0
+    elif cur.dtype == np.uint16:
+        dt = 1
+    else:
+        raise TypeError(cur.dtype)
+    rel = ctypes.c_double()
+    skip = ctypes.c_int32()
+    thr = float(np.float32(threshold))
+    rc = _load().oracle_fbc_rel_l1(_ptr(cur), _ptr(prev), cur.size, dt, thr,
+                                   ctypes.byref(rel), ctypes.byref(skip))
+    if rc != 0:
+        raise RuntimeError("oracle fbc failed")
+    return rel.value, int(skip.value)
+
+
+def channel_mean(x: np.ndarray) -> np.ndarray:
+    """[B, H, N, d] bf16 bits -> [B, H, d] fp32 means (fp64 sum, one rounding)."""
+    B, H, N, d = x.shape
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    out = np.empty((B, H, d), dtype=np.float32)
+    _load().oracle_channel_mean(_ptr(x), B * H, N, d, _ptr(out))
+    return out
+
+
+def quant_int8_blocks(x: np.ndarray, blk: int, mean: np.ndarray | None = None):
+    """Per-block INT8 codes [B,H,N,d] and scales [B,H,ceil(N/blk)] (fp32 mirror)."""
+    B, H, N, d = x.shape
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    nblk = (N + blk - 1) // blk
+    codes = np.empty((B, H, N, d), dtype=np.int8)
+    scales = np.empty((B, H, nblk), dtype=np.float32)
+    mp = None
+    if mean is not None:
+        mean = np.ascontiguousarray(mean, dtype=np.float32)
+        assert mean.shape == (B, H, d)
+        mp = _ptr(mean)
+    rc = _load().oracle_quant_int8_blocks(_ptr(x), B * H, N, d, blk, mp, _ptr(codes), _ptr(scales))
+    if rc != 0:
+        raise RuntimeError("oracle quant failed")
+    return codes, scales
+
+
+def quant_e4m3_channels(x: np.ndarray):
+    """Per-channel e4m3 codes [B,H,N,d] (uint8) and scales [B,H,d] (fp32 mirror)."""
+    B, H, N, d = x.shape
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    codes = np.empty((B, H, N, d), dtype=np.uint8)
+    scales = np.empty((B, H, d), dtype=np.float32)
+    _load().oracle_quant_e4m3_channels(_ptr(x), B * H, N, d, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    lib = _load()
+    flat = np.asarray(x, dtype=np.float32).reshape(-1)
+    return np.array([lib.oracle_e4m3_encode(float(t)) for t in flat], dtype=np.uint8).reshape(np.shape(x))
+
+
+def e4m3_decode(b: np.ndarray) -> np.ndarray:
+    lib = _load()
+    flat = np.asarray(b, dtype=np.uint8).reshape(-1)
+    return np.array([lib.oracle_e4m3_decode(int(t)) for t in flat], dtype=np.float32).reshape(np.shape(b))
+
+
+def emulated_q8_attention(q, k, v, scale: float | None = None, smooth_k: bool = True,
+                          rows=None) -> np.ndarray:
+    """fp64 attention over the dequantised 8-bit inputs (parity unpinned).
+
+    Replays the quantiser (Q per 128 tokens, K per 64 tokens after the optional
+    channel-mean subtraction, V per channel e4m3) and runs the exact fp64
+    attention on code * scale.  P's own rounding is not modelled.
+    """
+    B, H, N, d = q.shape
+    qc, qs = quant_int8_blocks(q, 128)
+    mean = channel_mean(k) if smooth_k else None
+    kc, ks = quant_int8_blocks(k, 64, mean)
+    vc, vs = quant_e4m3_channels(v)
+    tok = np.arange(N)
+    qd = qc.astype(np.float64) * qs[:, :, tok // 128, None].astype(np.float64)
+    kd = kc.astype(np.float64) * ks[:, :, tok // 64, None].astype(np.float64)
+    vd = e4m3_decode(vc).astype(np.float64) * vs[:, :, None, :].astype(np.float64)
+    return attention(qd, kd, vd, scale=scale, rows=rows)

@@ -1,0 +1,350 @@
+/*
+ * fp64 CPU oracle for the diffusion-transformer attention hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg may load this library.  It shares no code, header, table or
+ * constant with the CUDA library; it is deliberately plain, slow and written to
+ * be checked against the pages by eye.
+ *
+ * What it computes, and where the pages define it:
+ *
+ *  - Softmax attention O = softmax(s * Q K^T) V over the full, unmasked joint
+ *    token sequence.  "Flash Attention 2 accelerates Z-Image S3-DiT 6B"
+ *    (hotdry.top), opening section: text, visual-semantic and VAE tokens are
+ *    concatenated into one stream and attention computes QK^T, softmax and V;
+ *    the same operator is aten._scaled_dot_product_flash_attention in the FLOP
+ *    table of "TMAP image-to-video inference acceleration" (joto.ai), section
+ *    "hiding communication by reordering operators".  The pages print no
+ *    formula for the scale; s = 1/sqrt(d) (the scaled-dot-product default) is
+ *    passed in by the caller.  Two passes: the row maximum first, then the
+ *    exponentials, their sum, and the weighted sum of V, all in fp64.
+ *
+ *  - First-block-cache residual difference rel = sum|r_t - r_{t-1}| /
+ *    sum|r_{t-1}|, and the decision skip = rel < threshold.  "ParaAttention"
+ *    (diffusers docs), section "First Block Cache": the residual of the first
+ *    transformer block approximates the change of the model output; when the
+ *    difference is small enough, the cached residual is reused (0.08 is the
+ *    FLUX default).  Readings where the page is silent: strict "<" (at equality
+ *    the step is computed); a zero denominator gives rel = 0 when the
+ *    numerator is zero too, else +inf.
+ *
+ *  - The 8-bit quantiser of the attention inputs, in fp32 (so the GPU pre-pass
+ *    can be checked bit for bit).  "TMAP image-to-video inference
+ *    acceleration", section "optimising operator details": an all-zero channel
+ *    makes the quantisation scale zero and the division by it turns the output
+ *    to NaN; the fix guards that divide.  The block sizes (Q: 128 tokens,
+ *    K: 64 tokens), the optional K channel-mean subtraction and the FP8 e4m3
+ *    V are the workload's stated recipe; the pages only name per-block
+ *    quantisation ("128*128 per-block quantisation operator" in the same
+ *    section).  Readings: amax over the valid tokens of a block and all its
+ *    channels; inv = 127/amax and scale = amax/127 as fp32 divisions;
+ *    code = round-half-even(x*inv) clamped to [-127, 127]; amax == 0 gives
+ *    scale = inv = 0 and all-zero codes.  The K mean is summed in fp64 and
+ *    rounded to fp32, then subtracted in fp32.  V: per-channel amax over the
+ *    valid tokens, scale = amax/448, inv = 448/amax, the same zero guard.
+ *
+ *  - An FP8 E4M3 encoder written from the OCP 8-bit floating point
+ *    specification (bias 7, 3 mantissa bits, no infinities, 0x7F/0xFF NaN,
+ *    largest finite 448), round to nearest even, saturating to +-448.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* One query row against all N keys of one head.  k, v: [N, d] fp64. */
+static void attn_row(const double *qrow, const double *k, const double *v,
+                     int64_t N, int64_t d, double scale, double *logit, double *orow)
+{
+    double m = -INFINITY;
+    for (int64_t j = 0; j < N; ++j) {
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c)
+            dot += qrow[c] * k[j * d + c];
+        logit[j] = scale * dot;
+        if (logit[j] > m)
+            m = logit[j];
+    }
+    double l = 0.0;
+    for (int64_t c = 0; c < d; ++c)
+        orow[c] = 0.0;
+    for (int64_t j = 0; j < N; ++j) {
+        double w = exp(logit[j] - m);
+        l += w;
+        for (int64_t c = 0; c < d; ++c)
+            orow[c] += w * v[j * d + c];
+    }
+    for (int64_t c = 0; c < d; ++c)
+        orow[c] /= l;
+}
+
+/* Attention over fp64 inputs q, k, v: [B, H, N, d] contiguous.
+ * rows: query indices (nrows of them) or NULL for all N rows.
+ * o: [B, H, nrows, d] fp64 (nrows = N when rows == NULL). Returns 0 on success. */
+int oracle_attn_f64(const double *q, const double *k, const double *v, double *o,
+                    int64_t B, int64_t H, int64_t N, int64_t d, double scale,
+                    const int64_t *rows, int64_t nrows)
+{
+    if (N <= 0 || d <= 0)
+        return 1;
+    if (rows == NULL)
+        nrows = N;
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const double *kh = k + bh * N * d, *vh = v + bh * N * d;
+        int fail = 0;
+#pragma omp parallel
+        {
+            double *logit = (double *)malloc(sizeof(double) * (size_t)N);
+            if (!logit) {
+#pragma omp atomic write
+                fail = 1;
+            } else {
+#pragma omp for schedule(dynamic, 1)
+                for (int64_t r = 0; r < nrows; ++r) {
+                    int64_t i = rows ? rows[r] : r;
+                    attn_row(q + (bh * N + i) * d, kh, vh, N, d, scale, logit,
+                             o + (bh * nrows + r) * d);
+                }
+                free(logit);
+            }
+        }
+        if (fail)
+            return 2;
+    }
+    return 0;
+}
+
+/* Same, over bf16 inputs (uint16 bit patterns) widened exactly to fp64.
+ * Each head's K and V are widened once into fp64 scratch. */
+int oracle_attn_bf16in(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
+                       int64_t B, int64_t H, int64_t N, int64_t d, double scale,
+                       const int64_t *rows, int64_t nrows)
+{
+    if (N <= 0 || d <= 0)
+        return 1;
+    if (rows == NULL)
+        nrows = N;
+    double *kh = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    double *vh = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    double *qh = (double *)malloc(sizeof(double) * (size_t)(nrows * d));
+    if (!kh || !vh || !qh) {
+        free(kh); free(vh); free(qh);
+        return 2;
+    }
+    int fail = 0;
+    for (int64_t bh = 0; bh < B * H && !fail; ++bh) {
+#pragma omp parallel for schedule(static)
+        for (int64_t e = 0; e < N * d; ++e) {
+            kh[e] = bf16_to_double(k[bh * N * d + e]);
+            vh[e] = bf16_to_double(v[bh * N * d + e]);
+        }
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t i = rows ? rows[r] : r;
+            for (int64_t c = 0; c < d; ++c)
+                qh[r * d + c] = bf16_to_double(q[(bh * N + i) * d + c]);
+        }
+#pragma omp parallel
+        {
+            double *logit = (double *)malloc(sizeof(double) * (size_t)N);
+            if (!logit) {
+#pragma omp atomic write
+                fail = 1;
+            } else {
+#pragma omp for schedule(dynamic, 1)
+                for (int64_t r = 0; r < nrows; ++r)
+                    attn_row(qh + r * d, kh, vh, N, d, scale, logit, o + (bh * nrows + r) * d);
+                free(logit);
+            }
+        }
+    }
+    free(kh); free(vh); free(qh);
+    return fail ? 2 : 0;
+}
+
+/* First-block-cache residual difference.  dtype 0: fp32 values, 1: bf16 bits.
+ * Writes rel and skip (1 = reuse the cached residual). */
+int oracle_fbc_rel_l1(const void *cur, const void *prev, int64_t n, int dtype,
+                      double threshold, double *rel, int32_t *skip)
+{
+    double num = 0.0, den = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        double c, p;
+        if (dtype == 0) {
+            c = (double)((const float *)cur)[i];
+            p = (double)((const float *)prev)[i];
+        } else if (dtype == 1) {
+            c = bf16_to_double(((const uint16_t *)cur)[i]);
+            p = bf16_to_double(((const uint16_t *)prev)[i]);
+        } else {
+            return 1;
+        }
+        num += fabs(c - p);
+        den += fabs(p);
+    }
+    double r;
+    if (den > 0.0)
+        r = num / den;
+    else
+        r = (num > 0.0) ? INFINITY : 0.0;
+    *rel = r;
+    *skip = (r < threshold) ? 1 : 0;
+    return 0;
+}
+
+/* ---- 8-bit quantiser (fp32 arithmetic) -------------------------------- */
+
+/* Round half to even, then clamp to [-127, 127]. */
+static int8_t int8_code(float x)
+{
+    float r = nearbyintf(x); /* default rounding mode: to nearest, ties to even */
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    return (int8_t)r;
+}
+
+/* K channel means over the N tokens of each (b, h): mean[bh*d + c], summed in
+ * fp64 and rounded once to fp32. */
+int oracle_channel_mean(const uint16_t *x, int64_t BH, int64_t N, int64_t d, float *mean)
+{
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int64_t c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                s += bf16_to_double(x[(bh * N + n) * d + c]);
+            mean[bh * d + c] = (float)(s / (double)N);
+        }
+    return 0;
+}
+
+/* Per-block INT8 quantisation of x: [BH, N, d] bf16 bits.
+ * blk tokens per block; mean: [BH, d] fp32 subtracted first, or NULL.
+ * codes: [BH, N, d] int8; scales: [BH, ceil(N/blk)] fp32 (x ~ code * scale). */
+int oracle_quant_int8_blocks(const uint16_t *x, int64_t BH, int64_t N, int64_t d, int64_t blk,
+                             const float *mean, int8_t *codes, float *scales)
+{
+    if (blk <= 0)
+        return 1;
+    int64_t nblk = (N + blk - 1) / blk;
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int64_t b = 0; b < nblk; ++b) {
+            int64_t t0 = b * blk, t1 = t0 + blk < N ? t0 + blk : N;
+            float amax = 0.0f;
+            for (int64_t t = t0; t < t1; ++t)
+                for (int64_t c = 0; c < d; ++c) {
+                    float v = (float)bf16_to_double(x[(bh * N + t) * d + c]);
+                    if (mean)
+                        v = v - mean[bh * d + c];
+                    float a = fabsf(v);
+                    if (a > amax)
+                        amax = a;
+                }
+            float inv = 0.0f, scale = 0.0f;
+            if (amax > 0.0f) { /* zero-scale guard */
+                inv = 127.0f / amax;
+                scale = amax / 127.0f;
+            }
+            scales[bh * nblk + b] = scale;
+            for (int64_t t = t0; t < t1; ++t)
+                for (int64_t c = 0; c < d; ++c) {
+                    float v = (float)bf16_to_double(x[(bh * N + t) * d + c]);
+                    if (mean)
+                        v = v - mean[bh * d + c];
+                    codes[(bh * N + t) * d + c] = int8_code(v * inv);
+                }
+        }
+    return 0;
+}
+
+/* OCP FP8 E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits.  Normal
+ * values (1 + m/8) * 2^(e-7) for e in 1..15 (e = 15, m = 7 is NaN), subnormals
+ * (m/8) * 2^-6.  Round to nearest even; magnitudes past 448 saturate to 448. */
+uint8_t oracle_e4m3_encode(float x)
+{
+    if (isnan(x))
+        return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0)
+        return sign | 0x7E; /* satfinite */
+    if (a == 0.0)
+        return sign;
+    /* All e4m3 magnitudes are multiples of 2^-9; the quantum in the binade
+     * [2^e, 2^(e+1)) is 2^(e-3) for e >= -6, and 2^-9 below (subnormals). */
+    int e;
+    frexp(a, &e);          /* a = f * 2^e with f in [0.5, 1) -> binade 2^(e-1) */
+    int be = e - 1;
+    if (be < -6)
+        be = -6;
+    double quantum = ldexp(1.0, be - 3);
+    double q = a / quantum;                  /* exact: power-of-two divide */
+    double r = nearbyint(q);                 /* ties to even */
+    double y = r * quantum;
+    if (y >= 448.0)
+        return sign | 0x7E;
+    /* encode y */
+    if (y < ldexp(1.0, -6)) {                /* subnormal: m = y / 2^-9 */
+        int m = (int)(y / ldexp(1.0, -9));
+        return sign | (uint8_t)m;
+    }
+    int ye;
+    double yf = frexp(y, &ye);               /* y = yf * 2^ye, yf in [0.5,1) */
+    int expo = ye - 1 + 7;                   /* biased exponent */
+    int m = (int)((yf * 2.0 - 1.0) * 8.0);   /* exact */
+    return sign | (uint8_t)(expo << 3) | (uint8_t)m;
+}
+
+float oracle_e4m3_decode(uint8_t b)
+{
+    int s = b >> 7, e = (b >> 3) & 0xF, m = b & 7;
+    if (e == 15 && m == 7)
+        return NAN;
+    double v = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (float)(s ? -v : v);
+}
+
+/* Per-channel FP8 e4m3 quantisation of V: [BH, N, d] bf16 bits.
+ * codes: [BH, N, d] e4m3 bytes; scales: [BH, d] fp32 (v ~ e4m3(code) * scale). */
+int oracle_quant_e4m3_channels(const uint16_t *x, int64_t BH, int64_t N, int64_t d,
+                               uint8_t *codes, float *scales)
+{
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int64_t c = 0; c < d; ++c) {
+            float amax = 0.0f;
+            for (int64_t t = 0; t < N; ++t) {
+                float a = fabsf((float)bf16_to_double(x[(bh * N + t) * d + c]));
+                if (a > amax)
+                    amax = a;
+            }
+            float inv = 0.0f, scale = 0.0f;
+            if (amax > 0.0f) {
+                inv = 448.0f / amax;
+                scale = amax / 448.0f;
+            }
+            scales[bh * d + c] = scale;
+            for (int64_t t = 0; t < N; ++t) {
+                float v = (float)bf16_to_double(x[(bh * N + t) * d + c]);
+                codes[(bh * N + t) * d + c] = oracle_e4m3_encode(v * inv);
+            }
+        }
+    return 0;
+}
