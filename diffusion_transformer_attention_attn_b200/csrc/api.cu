@@ -1,0 +1,207 @@
+// C ABI of libditattn.so (declared in include/dit_attn.h): argument
+// validation, TMA tensor-map encoding and launches.  Host code only; the
+// arithmetic of every call runs in the kernels of attn_bf16.cu and
+// fbc_rel_l1.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "dit_attn.h"
+#include "internal.h"
+
+namespace ditk {
+
+// Device-side error word (one per device that loads the library); kernels
+// receive its address and write DIT_ERR_TIMEOUT there when a wait runs out.
+__device__ int g_dit_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    std::once_flag once;
+    cudaError_t init_err = cudaSuccess;
+    int* err_word = nullptr;
+    bool sm100 = false;
+};
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    return g_encode;
+}
+
+// Per-device set-up, done once with that device current: the address of the
+// error word and whether the device is an sm_100 part.
+DeviceState* device_state(dit_status* st) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        *st = DIT_ERR_CUDA;
+        return nullptr;
+    }
+    DeviceState& s = g_dev[dev];
+    std::call_once(s.once, [&s, dev] {
+        cudaDeviceProp prop;
+        s.init_err = cudaGetDeviceProperties(&prop, dev);
+        if (s.init_err != cudaSuccess) return;
+        s.sm100 = (prop.major == 10 && prop.minor == 0);
+        s.init_err = cudaGetSymbolAddress(reinterpret_cast<void**>(&s.err_word), g_dit_error);
+    });
+    if (s.init_err != cudaSuccess) {
+        *st = DIT_ERR_CUDA;
+        return nullptr;
+    }
+    if (!s.sm100) {
+        *st = DIT_ERR_UNSUPPORTED;
+        return nullptr;
+    }
+    *st = DIT_OK;
+    return &s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Byte ranges [p, p + span) of two tensors overlap?
+bool overlaps(const void* a, const void* b, int64_t span) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    const uintptr_t s = static_cast<uintptr_t>(span);
+    return x < y + s && y < x + s;
+}
+
+// Validation shared by the attention calls.  On success fills the strides.
+dit_status check_attn_args(const void* q, const void* k, const void* v, const void* o, int B, int H, int N, int d,
+                           const int64_t* strides, int64_t* sb, int64_t* sh, int64_t* sn) {
+    if (!q || !k || !v || !o) return DIT_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || N < 1 || d < 1) return DIT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DIT_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return DIT_ERR_UNSUPPORTED;
+    if (N > (1 << 30) || static_cast<int64_t>(B) * H > (1 << 24)) return DIT_ERR_UNSUPPORTED;
+    if (strides) {
+        *sb = strides[0];
+        *sh = strides[1];
+        *sn = strides[2];
+    } else {
+        *sn = d;
+        *sh = static_cast<int64_t>(N) * d;
+        *sb = static_cast<int64_t>(H) * N * d;
+    }
+    // TMA: every stride in bytes a multiple of 16, below 2^40; rows must not alias.
+    const int64_t st[3] = {*sb, *sh, *sn};
+    for (int i = 0; i < 3; ++i) {
+        if (st[i] <= 0 || (st[i] * 2) % 16 != 0 || st[i] * 2 >= (int64_t(1) << 40)) return DIT_ERR_INVALID_ARG;
+    }
+    if (*sn < d) return DIT_ERR_INVALID_ARG;
+    // Extent of one tensor in bytes (for the overlap check on o).
+    const int64_t span = ((B - 1) * *sb + (H - 1) * *sh + (N - 1) * *sn + d) * 2;
+    if (overlaps(o, q, span) || overlaps(o, k, span) || overlaps(o, v, span)) return DIT_ERR_INVALID_ARG;
+    return DIT_OK;
+}
+
+// 4-D map {d, N, H, B} over a bf16 tensor, box {64, 128, 1, 1}, 128-B swizzle.
+dit_status encode_bf16_map(CUtensorMap* map, const void* base, int B, int H, int N, int d, int64_t sb, int64_t sh,
+                           int64_t sn) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return DIT_ERR_CUDA;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(sn * 2), static_cast<cuuint64_t>(sh * 2),
+                                   static_cast<cuuint64_t>(sb * 2)};
+    const cuuint32_t box[4] = {64, 128, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_INVALID_ARG;
+}
+
+float default_scale(int d) { return 1.0f / std::sqrt(static_cast<float>(d)); }
+
+}  // namespace
+}  // namespace ditk
+
+using namespace ditk;
+
+extern "C" {
+
+dit_status dit_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                        const int64_t* strides, float scale, void* stream) {
+    int64_t sb, sh, sn;
+    dit_status st = check_attn_args(q, k, v, o, B, H, N, d, strides, &sb, &sh, &sn);
+    if (st != DIT_OK) return st;
+    if (!(scale == scale) || std::isinf(scale)) return DIT_ERR_INVALID_ARG;
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    CUtensorMap tq, tk, tv;
+    if ((st = encode_bf16_map(&tq, q, B, H, N, d, sb, sh, sn)) != DIT_OK) return st;
+    if ((st = encode_bf16_map(&tk, k, B, H, N, d, sb, sh, sn)) != DIT_OK) return st;
+    if ((st = encode_bf16_map(&tv, v, B, H, N, d, sb, sh, sn)) != DIT_OK) return st;
+    const float s = scale > 0.f ? scale : default_scale(d);
+    const float scale_log2 = static_cast<float>(static_cast<double>(s) * 1.4426950408889634);
+    cudaError_t e = launch_attn_bf16(tq, tk, tv, o, sb, sh, sn, B, H, N, d, scale_log2, ds->err_word,
+                                     static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+size_t fbc_rel_l1_workspace_bytes(int64_t n) { return n < 1 ? 0 : fbc_workspace_bytes(n); }
+
+dit_status fbc_rel_l1(const void* r_cur, const void* r_prev, int64_t n, int dtype, float threshold, double* out_rel,
+                      int32_t* out_skip, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!r_cur || !r_prev || !out_rel || !out_skip || n < 1) return DIT_ERR_INVALID_ARG;
+    if (dtype != DIT_DTYPE_F32 && dtype != DIT_DTYPE_BF16) return DIT_ERR_INVALID_ARG;
+    if (!aligned16(r_cur) || !aligned16(r_prev)) return DIT_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out_rel) & 7u) != 0 || (reinterpret_cast<uintptr_t>(out_skip) & 3u) != 0)
+        return DIT_ERR_INVALID_ARG;
+    if (!(threshold == threshold)) return DIT_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < fbc_workspace_bytes(n)) return DIT_ERR_WORKSPACE;
+    dit_status st;
+    if (!device_state(&st)) return st;
+    cudaError_t e = launch_fbc_rel_l1(r_cur, r_prev, n, dtype, threshold, out_rel, out_skip, workspace,
+                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+dit_status dit_get_device_status(void* stream) {
+    dit_status st;
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DIT_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_dit_error, sizeof(int)) != cudaSuccess) return DIT_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_dit_error, &zero, sizeof(int)) != cudaSuccess) return DIT_ERR_CUDA;
+        return static_cast<dit_status>(word);
+    }
+    return DIT_OK;
+}
+
+const char* dit_status_string(int status) {
+    switch (status) {
+        case DIT_OK: return "DIT_OK";
+        case DIT_ERR_INVALID_ARG: return "DIT_ERR_INVALID_ARG";
+        case DIT_ERR_UNSUPPORTED: return "DIT_ERR_UNSUPPORTED";
+        case DIT_ERR_WORKSPACE: return "DIT_ERR_WORKSPACE";
+        case DIT_ERR_CUDA: return "DIT_ERR_CUDA";
+        case DIT_ERR_TIMEOUT: return "DIT_ERR_TIMEOUT";
+        default: return "DIT_ERR_UNKNOWN";
+    }
+}
+
+}  // extern "C"

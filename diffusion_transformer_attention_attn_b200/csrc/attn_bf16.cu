@@ -1,0 +1,432 @@
+// Softmax attention O = softmax(scale · Q Kᵀ) V for bf16 [B, H, N, d] tensors
+// on sm_100a: TMA-staged tiles, tcgen05 MMAs accumulating in tensor memory,
+// and an exp2 online softmax with a running row max and row sum.
+//
+// What is computed follows "Flash Attention 2 accelerates Z-Image S3-DiT 6B"
+// (opening section): one joint token stream, no mask, QKᵀ, softmax and V
+// evaluated tile by tile in on-chip memory so the N×N logits never reach HBM.
+//
+// Work unit: one CTA takes 256 query rows (two 128-row tiles, "Q0" and "Q1")
+// of one (b, h) and sweeps all keys in 128-key tiles.  Warp roles:
+//   warps 0-3  softmax for Q0 (one thread per query row)
+//   warps 4-7  softmax for Q1
+//   warp  8    TMA producer (Q once, then a ring of K and V tiles)
+//   warp  9    MMA issuer (one elected lane)
+// Tensor memory (512 columns × 128 lanes × 32 bit):
+//   [0,128)  S0 = Q0·Kᵀ (fp32); after the softmax, P0 (bf16 pairs) in [0,64)
+//   [128,256) S1 / P1
+//   [256,256+d) O0 accumulator;  [256+d, 256+2d) O1 accumulator
+// The MMA warp alternates the two tiles so that the tensor core computes
+// P1·V and the next Q1·Kᵀ while the Q0 softmax runs, and vice versa.
+//
+// Online softmax (per row, in log2 units t = s·scale·log2 e): the running max
+// m only moves when a new tile's max exceeds it by more than 8 (a factor 256
+// in P); only then is the O row in tensor memory rescaled by 2^(m_old-m_new)
+// and the row sum l with it.  P = 2^(t - m) ≤ 256 is exact enough in bf16
+// and O, l are fp32.  Keys at or past N (the ragged last tile, zero-filled
+// by TMA) get t = -inf, hence P = 0.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace ditk {
+namespace {
+
+constexpr int kBM = 128;          // query rows per tile
+constexpr int kBN = 128;          // keys per tile
+constexpr int kThreads = 320;     // 10 warps
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kHalfBytes = 128 * 128;  // one TMA box: 128 rows × 64 bf16 (128 B, swizzled)
+
+template <int D>
+struct Cfg {
+    static constexpr int kTileBytes = kBM * D * 2;            // 128 rows × d bf16
+    static constexpr int kHalves = D / 64;                    // 64-element swizzle atoms along d
+    static constexpr int kStages = (D == 128) ? 2 : 4;        // K ring depth == V ring depth
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = 2 * kTileBytes;
+    static constexpr int kVOff = kKOff + kStages * kTileBytes;
+    static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+    // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
+    //           s_full[2], p_full[2], o_ready[2], mma_done
+    static constexpr int kNumBars = 1 + 4 * kStages + 6 + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 64 + 1024;    // + slack for 1024-B alignment
+    // S tiles: M=128 rows, N=128 keys, K-major A (Q) and B (K).
+    static constexpr uint32_t kIdescQK = make_idesc(1, 1, 1, 0, 0, 128, kBN);
+    // O += P·V: A = P from TMEM (K-major), B = V with d contiguous (MN-major).
+    static constexpr uint32_t kIdescPV = make_idesc(1, 1, 1, 0, 1, 128, D);
+};
+
+struct Bars {
+    uint64_t* q_full;
+    uint64_t* k_full;
+    uint64_t* k_empty;
+    uint64_t* v_full;
+    uint64_t* v_empty;
+    uint64_t* s_full;
+    uint64_t* p_full;
+    uint64_t* o_ready;
+    uint64_t* mma_done;
+};
+
+template <int D>
+__device__ __forceinline__ Bars carve_bars(uint8_t* base) {
+    using C = Cfg<D>;
+    uint64_t* b = reinterpret_cast<uint64_t*>(base + C::kBarOff);
+    Bars r;
+    r.q_full = b;
+    r.k_full = b + 1;
+    r.k_empty = r.k_full + C::kStages;
+    r.v_full = r.k_empty + C::kStages;
+    r.v_empty = r.v_full + C::kStages;
+    r.s_full = r.v_empty + C::kStages;
+    r.p_full = r.s_full + 2;
+    r.o_ready = r.p_full + 2;
+    r.mma_done = r.o_ready + 2;
+    return r;
+}
+
+// K-major operand (Q or K tile) for k-step kk (16 bf16 along d): the d-halves
+// are separate 16 KB swizzle panels; inside a panel, +32 B per k-step.
+template <int D>
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_saddr, int kk) {
+    const uint32_t a = tile_saddr + (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    return smem_desc_sw128(a, 16, 1024);
+}
+// MN-major V tile for key-step kk (16 keys): +16 rows × 128 B per step;
+// LBO = distance between the 64-wide d panels, SBO = 8 keys × 128 B.
+__device__ __forceinline__ uint64_t desc_v(uint32_t tile_saddr, int kk) {
+    return smem_desc_sw128(tile_saddr + kk * 16 * 128, kHalfBytes, 1024);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                         const __grid_constant__ CUtensorMap tv, __nv_bfloat16* __restrict__ o, int64_t sb,
+                         int64_t sh, int64_t sn, int H, int N, int n_pairs, float scale_log2, int* err) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const Bars bars = carve_bars<D>(smem);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const int pair = blockIdx.x % n_pairs;
+    const int bh = blockIdx.x / n_pairs;
+    const int b = bh / H;
+    const int h = bh % H;
+    const int q0 = pair * 2 * kBM;
+    const int nkv = (N + kBN - 1) / kBN;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bars.q_full, 1);
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&bars.k_full[s], 1);
+            mbar_init(&bars.k_empty[s], 1);
+            mbar_init(&bars.v_full[s], 1);
+            mbar_init(&bars.v_empty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars.s_full[t], 1);
+            mbar_init(&bars.p_full[t], kBM);
+            mbar_init(&bars.o_ready[t], 1);
+        }
+        mbar_init(bars.mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t smem_base = smem_u32(smem);
+
+    if (warp == kLoadWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tq);
+            tma_prefetch_desc(&tk);
+            tma_prefetch_desc(&tv);
+            mbar_arrive_expect_tx(bars.q_full, 2 * C::kTileBytes);
+            for (int t = 0; t < 2; ++t)
+                for (int hf = 0; hf < C::kHalves; ++hf)
+                    tma_load_4d(smem + C::kQOff + t * C::kTileBytes + hf * kHalfBytes, &tq, bars.q_full, hf * 64,
+                                q0 + t * kBM, h, b);
+        }
+        __syncwarp();
+        int nk[C::kStages], nv[C::kStages];  // times each stage was armed
+#pragma unroll
+        for (int s = 0; s < C::kStages; ++s) nk[s] = nv[s] = 0;
+        for (int j = 0; j < nkv; ++j) {
+            const int s = j % C::kStages;
+            const uint32_t ph = (j / C::kStages) & 1;
+            if (j >= C::kStages && !mbar_wait(&bars.k_empty[s], ph ^ 1, abort_flag, err)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars.k_full[s], C::kTileBytes);
+                for (int hf = 0; hf < C::kHalves; ++hf)
+                    tma_load_4d(smem + C::kKOff + s * C::kTileBytes + hf * kHalfBytes, &tk, &bars.k_full[s],
+                                hf * 64, j * kBN, h, b);
+            }
+            __syncwarp();
+            ++nk[s];
+            if (j >= C::kStages && !mbar_wait(&bars.v_empty[s], ph ^ 1, abort_flag, err)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars.v_full[s], C::kTileBytes);
+                for (int hf = 0; hf < C::kHalves; ++hf)
+                    tma_load_4d(smem + C::kVOff + s * C::kTileBytes + hf * kHalfBytes, &tv, &bars.v_full[s],
+                                hf * 64, j * kBN, h, b);
+            }
+            __syncwarp();
+            ++nv[s];
+        }
+        if (*abort_flag && lane == 0) {
+            // Let every copy this warp started land before the CTA can exit:
+            // the n-th arming of a stage completes that barrier's phase n-1.
+            mbar_wait_drain(bars.q_full, 0);
+            for (int s = 0; s < C::kStages; ++s) {
+                if (nk[s] > 0) mbar_wait_drain(&bars.k_full[s], (nk[s] - 1) & 1);
+                if (nv[s] > 0) mbar_wait_drain(&bars.v_full[s], (nv[s] - 1) & 1);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t sQ0 = smem_base + C::kQOff;
+        const uint32_t sQ1 = sQ0 + C::kTileBytes;
+        const uint32_t tS0 = tmem, tS1 = tmem + 128;
+        const uint32_t tO0 = tmem + 256, tO1 = tmem + 256 + D;
+        bool ok = mbar_wait(bars.q_full, 0, abort_flag, err) && mbar_wait(&bars.k_full[0], 0, abort_flag, err);
+        if (ok) {
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t sK = smem_base + C::kKOff;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16_ss(tS0, desc_kmajor<D>(sQ0, kk), desc_kmajor<D>(sK, kk), C::kIdescQK, kk > 0);
+                mma_commit(&bars.s_full[0]);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16_ss(tS1, desc_kmajor<D>(sQ1, kk), desc_kmajor<D>(sK, kk), C::kIdescQK, kk > 0);
+                mma_commit(&bars.s_full[1]);
+                mma_commit(&bars.k_empty[0]);
+            }
+            __syncwarp();
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int vs = j % C::kStages;
+                const uint32_t sV = smem_base + C::kVOff + vs * C::kTileBytes;
+                const bool more = j + 1 < nkv;
+                const int ks = (j + 1) % C::kStages;
+                const uint32_t sK = smem_base + C::kKOff + ks * C::kTileBytes;
+                ok = mbar_wait(&bars.v_full[vs], (j / C::kStages) & 1, abort_flag, err) &&
+                     mbar_wait(&bars.p_full[0], j & 1, abort_flag, err);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_bf16_ts(tO0, tS0 + kk * 8, desc_v(sV, kk), C::kIdescPV, (j > 0 || kk > 0));
+                    mma_commit(&bars.o_ready[0]);
+                }
+                __syncwarp();
+                if (more) {
+                    ok = mbar_wait(&bars.k_full[ks], ((j + 1) / C::kStages) & 1, abort_flag, err);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_bf16_ss(tS0, desc_kmajor<D>(sQ0, kk), desc_kmajor<D>(sK, kk), C::kIdescQK, kk > 0);
+                        mma_commit(&bars.s_full[0]);
+                    }
+                    __syncwarp();
+                }
+                ok = mbar_wait(&bars.p_full[1], j & 1, abort_flag, err);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_bf16_ts(tO1, tS1 + kk * 8, desc_v(sV, kk), C::kIdescPV, (j > 0 || kk > 0));
+                    mma_commit(&bars.o_ready[1]);
+                    mma_commit(&bars.v_empty[vs]);
+                    if (more) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_bf16_ss(tS1, desc_kmajor<D>(sQ1, kk), desc_kmajor<D>(sK, kk), C::kIdescQK, kk > 0);
+                        mma_commit(&bars.s_full[1]);
+                        mma_commit(&bars.k_empty[ks]);
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        // Every MMA issued above has completed once mma_done flips.
+        if (lane == 0) {
+            mma_commit(bars.mma_done);
+            mbar_wait_drain(bars.mma_done, 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax (warps 0-7)
+        const int wg = warp >> 2;  // which query tile
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + wg * 128;
+        const uint32_t tO = tmem + lane_off + 256 + wg * D;
+        float m = -INFINITY;
+        float l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nkv; ++j) {
+            ok = mbar_wait(&bars.s_full[wg], j & 1, abort_flag, err);
+            if (!ok) break;
+            tc_fence_after();
+            float x[kBN];
+            {
+                uint32_t r[kBN / 32][32];
+#pragma unroll
+                for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, r[c]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < kBN / 32; ++c) {
+                    reg_fence32(r[c]);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[c][i]);
+                }
+            }
+            if (j == nkv - 1) {
+                const int valid = N - j * kBN;
+                if (valid < kBN) {
+#pragma unroll
+                    for (int c = 0; c < kBN; ++c)
+                        if (c >= valid) x[c] = -INFINITY;
+                }
+            }
+            // Row max over the tile (tree of independent fmax).
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = x[i];
+#pragma unroll
+            for (int c = 8; c < kBN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+            const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float m_new = fmaxf(m, tmax * scale_log2);
+            if (j == 0) {
+                m = m_new;
+            } else {
+                const bool need = m_new > m + 8.0f;
+                if (__any_sync(0xffffffffu, need)) {
+                    // O holds P_{<j}·V; rescale it once P_{j-1}·V has landed.
+                    ok = mbar_wait(&bars.o_ready[wg], (j - 1) & 1, abort_flag, err);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
+                    uint32_t r[32];
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        tmem_ld32(tO + c * 32, r);
+                        tmem_wait_ld();
+                        reg_fence32(r);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st32(tO + c * 32, r);
+                    }
+                    tmem_wait_st();
+                    if (need) {
+                        l *= alpha;
+                        m = m_new;
+                    }
+                }
+            }
+            const float negm = -m;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t p[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float a = ex2_approx(fmaf(x[c * 64 + 2 * i], scale_log2, negm));
+                    const float bb = ex2_approx(fmaf(x[c * 64 + 2 * i + 1], scale_log2, negm));
+                    ls[i & 3] += a + bb;
+                    p[i] = pack_bf16x2(a, bb);
+                }
+                tmem_st32(tS + c * 32, p);
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars.p_full[wg]);
+        }
+        // Epilogue: O / l -> bf16 -> global (rows at or past N are padding).
+        if (ok) ok = mbar_wait(&bars.o_ready[wg], (nkv - 1) & 1, abort_flag, err);
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = 1.0f / l;
+            const int qrow = q0 + wg * kBM + row;
+            __nv_bfloat16* orow = o + b * sb + h * sh + static_cast<int64_t>(qrow) * sn;
+            uint32_t r[32];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                tmem_ld32(tO + c * 32, r);
+                tmem_wait_ld();
+                reg_fence32(r);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+                if (qrow < N) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int64_t sb,
+                     int64_t sh, int64_t sn, int B, int H, int N, float scale_log2, int* err, cudaStream_t stream) {
+    using C = Cfg<D>;
+    static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int n_qt = (N + kBM - 1) / kBM;
+    const int n_pairs = (n_qt + 1) / 2;
+    const int64_t grid = static_cast<int64_t>(B) * H * n_pairs;
+    if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    attn_fwd_bf16_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(
+        tq, tk, tv, static_cast<__nv_bfloat16*>(o), sb, sh, sn, H, N, n_pairs, scale_log2, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                             int64_t sb, int64_t sh, int64_t sn, int B, int H, int N, int d, float scale_log2,
+                             int* err, cudaStream_t stream) {
+    if (d == 128) return launch_d<128>(tq, tk, tv, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
+    if (d == 64) return launch_d<64>(tq, tk, tv, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace ditk

@@ -1,0 +1,114 @@
+/*
+ * dit_attn.h — C ABI of the B200 (sm_100a) diffusion-transformer attention
+ * library (libditattn.so).
+ *
+ * The library holds the hot path of image and video diffusion transformers:
+ * full bidirectional multi-head self-attention over one joint token stream,
+ * and the first-block-cache residual difference that decides whether a
+ * denoising step may reuse its cached residual.
+ *
+ * Conventions shared by every entry point
+ *   - Every buffer is caller-owned device memory.  The library allocates no
+ *     device memory on any call; where a kernel needs scratch, the caller
+ *     passes a workspace whose size the matching *_workspace_bytes call gives.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *     is the legacy default stream).  Argument errors are reported before any
+ *     launch and leave every output untouched.
+ *   - A launch failure returns DIT_ERR_CUDA.  Every wait inside a kernel is
+ *     bounded in time: a wait that runs out records DIT_ERR_TIMEOUT in a
+ *     device-side error word instead of hanging, and dit_get_device_status
+ *     reports (and clears) it.
+ *   - NaN or Inf inputs are outside the contract.
+ */
+#ifndef DIT_ATTN_H
+#define DIT_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DIT_OK = 0,
+    DIT_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or stride */
+    DIT_ERR_UNSUPPORTED = 2, /* valid request this build does not serve (e.g. d = 96) */
+    DIT_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
+    DIT_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed */
+    DIT_ERR_TIMEOUT = 5      /* a device-side wait ran out (see dit_get_device_status) */
+} dit_status;
+
+typedef enum { DIT_DTYPE_F32 = 0, DIT_DTYPE_BF16 = 1 } dit_dtype;
+
+/*
+ * dit_attn_fwd — softmax attention O = softmax(scale · Q Kᵀ) V, per (b, h),
+ * over all N keys (no mask: the text and visual tokens form one joint,
+ * bidirectional stream).
+ *
+ * Defined by: "Flash Attention 2 accelerates Z-Image S3-DiT 6B" (hotdry.top),
+ * opening section (text, visual and VAE tokens concatenated into a single
+ * stream; attention computed as QKᵀ, softmax, V in on-chip tiles), and by the
+ * FLOP table of "TMAP image-to-video inference acceleration" (joto.ai),
+ * section on hiding communication, where this operator
+ * (aten._scaled_dot_product_flash_attention) is about 74% of all FLOPs.
+ *
+ *   q, k, v  device bf16, logical shape [B, H, N, d], d contiguous (stride 1).
+ *   o        device bf16 output, same shape; its strides are `strides` too.
+ *   strides  element strides of dimensions (b, h, n), shared by q, k, v, o;
+ *            NULL means contiguous [B, H, N, d].  Each stride × 2 bytes must
+ *            be a multiple of 16.
+ *   d        64 or 128 (others: DIT_ERR_UNSUPPORTED).
+ *   scale    logit scale; scale <= 0 means 1/sqrt(d) (computed in fp32).
+ *   Pointers must be 16-byte aligned.  B, H, N >= 1.
+ *   o must not overlap q, k or v.  Accumulation is fp32; O is rounded to
+ *   bf16 (round to nearest even).
+ */
+dit_status dit_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                        int B, int H, int N, int d, const int64_t* strides,
+                        float scale, void* stream);
+
+/*
+ * fbc_rel_l1 — first-block-cache residual difference and decision:
+ *   rel  = Σ|r_cur − r_prev| / Σ|r_prev|   (over all n elements)
+ *   skip = rel < threshold                 (1: reuse the cached residual)
+ *
+ * Defined by: "ParaAttention" (diffusers docs), section "First Block Cache":
+ * the residual of the first transformer block between consecutive steps
+ * approximates the change of the model output; when it is small enough
+ * (0.08 for FLUX), the remaining blocks are skipped and the cache is reused.
+ * Readings where the page is silent: the comparison is strict (at equality
+ * the step is computed); Σ|r_prev| = 0 gives rel = 0 when the numerator is 0
+ * too, else +inf.
+ *
+ *   r_cur, r_prev  device arrays of n elements of `dtype` (fp32 or bf16),
+ *                  16-byte aligned.  n >= 1.
+ *   out_rel        device double[1];  out_skip  device int32[1].
+ *   workspace      device memory of fbc_rel_l1_workspace_bytes(n) bytes,
+ *                  16-byte aligned, zero-filled before its first use; each
+ *                  call leaves it zero-filled again.  Calls that share one
+ *                  workspace must be ordered (same stream, or synchronised).
+ *   Partial sums are fp32 per thread and fp64 across threads and blocks, in a
+ *   fixed order: the result is deterministic for a given n.
+ */
+size_t fbc_rel_l1_workspace_bytes(int64_t n);
+dit_status fbc_rel_l1(const void* r_cur, const void* r_prev, int64_t n, int dtype,
+                      float threshold, double* out_rel, int32_t* out_skip,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * dit_get_device_status — synchronises `stream`, then returns and clears the
+ * device-side error word of the current device (DIT_ERR_TIMEOUT if a bounded
+ * wait inside a kernel ran out since the last call), or DIT_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+dit_status dit_get_device_status(void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* dit_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIT_ATTN_H */

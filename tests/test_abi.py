@@ -1,0 +1,111 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments with the documented status before
+touching the device (no GPU is needed for any of these)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import diffusion_transformer_attention_attn_b200 as dit
+from diffusion_transformer_attention_attn_b200 import build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return dit.load_library()
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M):
+            if m.group(1) not in ("if", "defined"):
+                names.append(m.group(1))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for expected in ("dit_attn_fwd", "fbc_rel_l1", "fbc_rel_l1_workspace_bytes", "dit_get_device_status",
+                     "dit_status_string"):
+        assert expected in names
+    assert set(names) == set(dit.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert dit.status_string(0) == "DIT_OK"
+    assert dit.status_string(5) == "DIT_ERR_TIMEOUT"
+    assert dit.status_string(99) == "DIT_ERR_UNKNOWN"
+
+
+# Fake, 16-byte-aligned, non-overlapping "device" addresses: every case below
+# is rejected during validation, before any pointer is used.
+Q, K, V, O = 0x10000000, 0x20000000, 0x30000000, 0x40000000
+
+
+def _attn(lib, q=Q, k=K, v=V, o=O, B=1, H=2, N=256, d=64, strides=None, scale=0.0):
+    st = None
+    if strides is not None:
+        st = (ctypes.c_int64 * 3)(*strides)
+    return lib.dit_attn_fwd(q, k, v, o, B, H, N, d, st, scale, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=0), dit.DIT_ERR_INVALID_ARG),
+    (dict(o=0), dit.DIT_ERR_INVALID_ARG),
+    (dict(N=0), dit.DIT_ERR_INVALID_ARG),
+    (dict(B=0), dit.DIT_ERR_INVALID_ARG),
+    (dict(H=-1), dit.DIT_ERR_INVALID_ARG),
+    (dict(d=96), dit.DIT_ERR_UNSUPPORTED),
+    (dict(d=256), dit.DIT_ERR_UNSUPPORTED),
+    (dict(k=K + 8), dit.DIT_ERR_INVALID_ARG),            # misaligned
+    (dict(o=Q + 64), dit.DIT_ERR_INVALID_ARG),           # output overlaps q
+    (dict(strides=(256 * 64 * 2, 256 * 64, 60)), dit.DIT_ERR_INVALID_ARG),  # row stride < d
+    (dict(strides=(256 * 64 * 2, 256 * 64, 68)), dit.DIT_ERR_INVALID_ARG),  # 136 B: not a multiple of 16
+    (dict(scale=float("nan")), dit.DIT_ERR_INVALID_ARG),
+])
+def test_attn_argument_errors(lib, kw, status):
+    assert _attn(lib, **kw) == status
+
+
+def test_fbc_argument_errors(lib):
+    n = 1000
+    ws = lib.fbc_rel_l1_workspace_bytes(n)
+    assert ws >= 16
+    assert lib.fbc_rel_l1_workspace_bytes(0) == 0
+    call = lambda **kw: lib.fbc_rel_l1(kw.get("cur", Q), kw.get("prev", K), kw.get("n", n), kw.get("dtype", 0),
+                                       kw.get("thr", 0.08), kw.get("rel", V), kw.get("skip", V + 64),
+                                       kw.get("ws", O), kw.get("wsb", ws), None)
+    assert call(cur=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(n=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(dtype=7) == dit.DIT_ERR_INVALID_ARG
+    assert call(prev=K + 4) == dit.DIT_ERR_INVALID_ARG
+    assert call(rel=V + 4) == dit.DIT_ERR_INVALID_ARG
+    assert call(thr=float("nan")) == dit.DIT_ERR_INVALID_ARG
+    assert call(ws=0) == dit.DIT_ERR_WORKSPACE
+    assert call(wsb=ws - 1) == dit.DIT_ERR_WORKSPACE
+    assert call(ws=O + 8) == dit.DIT_ERR_WORKSPACE
+
+
+def test_product_path_does_not_reach_the_oracle():
+    # The binding and the library sources never name the oracle.
+    pkg = os.path.join(ROOT, "diffusion_transformer_attention_attn_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "liboracle" not in text, f
