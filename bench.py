@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Throughput of the diffusion-transformer attention hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input of
+the long-video workload (HunyuanVideo 720p x 129 frames: B=1, H=24,
+N=119056 joint tokens, d=128, bf16 Q/K/V ~ N(0,1) with K per-channel offsets
+~ N(0, 2^2)):
+  * dit_attn_fwd  — bf16 softmax attention over all 119056 keys
+  * fbc_rel_l1    — first-block-cache decision over that model's residual pair
+                    (119056 x 3072 bf16, drift N(0, 0.03^2), threshold 0.08)
+
+The metric is attention TFLOP/s (4*B*H*N^2*d per attention call) over the
+whole step.  Inputs (2.2 GB of Q/K/V, 1.5 GB of residuals) are far larger than
+the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica of the workload (weak
+scaling; no data-path collective), timed as the max over ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from diffusion_transformer_attention_attn_b200 import inputs  # noqa: E402
+
+METRIC = "attention TFLOPS (4·B·H·N²·d/s) and % of B200 tensor peak at N=119k, bf16 & 8-bit"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                if self.uuid and self.uuid not in parts[1]:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
+        pw = [num(r[4]) for r in rows if num(r[4]) is not None]
+        # samples under load: power above the midpoint of the range seen
+        load = sm
+        if pw and max(pw) > 0:
+            thr = min(pw) + 0.5 * (max(pw) - min(pw))
+            load = [num(r[2]) for r in rows if num(r[4]) is not None and num(r[4]) >= thr and num(r[2])]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def pinned_bf16(bits: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+
+
+def cpu_info():
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model
+
+
+def time_oracle(case: inputs.AttnCase, q, k, v, fbc_case, cur, prev, rows_per_head: int):
+    """One bounded oracle step: sampled query rows of every head against all
+    keys, plus the residual difference over the same token rows."""
+    import oracle
+    rows = inputs.sample_rows(case.N, rows_per_head, seed=7)
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, rows=rows)
+    r = rows
+    oracle.fbc_rel_l1(cur[r], prev[r], fbc_case.threshold)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * case.B * case.H * len(rows) * case.N * case.d
+    return dt, flops, len(rows)
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+# The timed workload (default) and two smaller ones of the same shape family
+# used for profiling captures.  Each step's residual pair is tokens x (H*d).
+WORKLOADS = {
+    "video_long": inputs.VIDEO_LONG,
+    "video_mid": inputs.VIDEO_MID,
+    "image": inputs.IMAGE,
+}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    case = WORKLOADS[args.workload]
+    fcase = inputs.FbcCase(f"fbc_{case.N}x{case.H * case.d}_bf16", case.N, case.H * case.d, "bf16", 0.03, 0.08)
+    q, k, v = inputs.attn_inputs(case)
+    cur, prev = inputs.fbc_inputs(fcase)
+    cores = oracle.num_threads()
+    rows_per_head = args.ref_rows
+    for _ in range(args.warmup):
+        time_oracle(case, q, k, v, fcase, cur, prev, max(2, rows_per_head // 8))
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl, nr = time_oracle(case, q, k, v, fcase, cur, prev, rows_per_head)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = (f"{nr} query rows per head x {case.H} heads against all {case.N} keys, plus the "
+              f"residual difference over the same {nr} token rows x {fcase.cols}, per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": case.name, "B": case.B, "H": case.H, "N": case.N, "d": case.d},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                         "cpu": cpu_info()},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import diffusion_transformer_attention_attn_b200 as dit
+
+    ws, rank, local = dist_env()
+    if ws != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={ws}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    dit.load_library()
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    base = WORKLOADS[args.workload]
+    case = inputs.AttnCase(base.name, base.B, base.H, base.N, base.d, k_offset_std=base.k_offset_std, seed=rank)
+    fcase = inputs.FbcCase(f"fbc_{base.N}x{base.H * base.d}_bf16", base.N, base.H * base.d, "bf16", 0.03, 0.08,
+                           seed=rank)
+    q, k, v = inputs.attn_inputs(case)
+    cur, prev = inputs.fbc_inputs(fcase)
+
+    hq, hk, hv = (pinned_bf16(t) for t in (q, k, v))
+    hcur, hprev = pinned_bf16(cur), pinned_bf16(prev)
+    ho = torch.empty_like(hq).pin_memory()
+    hrel = torch.empty(1, dtype=torch.float64).pin_memory()
+    hskip = torch.empty(1, dtype=torch.int32).pin_memory()
+    del q, k, v, cur, prev
+
+    dq, dk, dv = (t.to(dev) for t in (hq, hk, hv))
+    do = torch.empty_like(dq)
+    dcur, dprev = hcur.to(dev), hprev.to(dev)
+    drel = torch.empty(1, dtype=torch.float64, device=dev)
+    dskip = torch.empty(1, dtype=torch.int32, device=dev)
+    fws = dit.fbc_workspace(dcur.numel(), dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    launches_per_step = 2  # attention + residual difference
+
+    def step():
+        dit.dit_attn_fwd(dq, dk, dv, o=do)
+        dit.fbc_rel_l1(dcur, dprev, fcase.threshold, out_rel=drel, out_skip=dskip, workspace=fws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = dit.dit_get_device_status()
+    if st != 0:
+        raise SystemExit(f"device status after warm-up: {dit.status_string(st)}")
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+
+    # ---- device-resident timed region
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ef = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    ev[0].record(stream)
+    for i in range(K):
+        ea[i][0].record(stream)
+        dit.dit_attn_fwd(dq, dk, dv, o=do)
+        ea[i][1].record(stream)
+        ef[i][0].record(stream)
+        dit.fbc_rel_l1(dcur, dprev, fcase.threshold, out_rel=drel, out_skip=dskip, workspace=fws)
+        ef[i][1].record(stream)
+    ev[1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    ms = ev[0].elapsed_time(ev[1])
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ea)
+    fbc_ms = statistics.mean(a.elapsed_time(b) for a, b in ef)
+    st = dit.dit_get_device_status()
+    if st != 0:
+        raise SystemExit(f"device status after timing: {dit.status_string(st)}")
+
+    # ---- end-to-end through the public API from pinned host buffers
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    e1[0].record(stream)
+    for _ in range(K):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dit.dit_attn_fwd(dq, dk, dv, o=do)
+        ho.copy_(do, non_blocking=True)
+        dcur.copy_(hcur, non_blocking=True)
+        dprev.copy_(hprev, non_blocking=True)
+        dit.fbc_rel_l1(dcur, dprev, fcase.threshold, out_rel=drel, out_skip=dskip, workspace=fws)
+        hrel.copy_(drel, non_blocking=True)
+        hskip.copy_(dskip, non_blocking=True)
+    e1[1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e1[0].elapsed_time(e1[1])
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcur, hprev))
+    d2h = ho.numel() * ho.element_size() + 8 + 4
+
+    # ---- max over ranks
+    t = torch.tensor([ms, e2e_ms, attn_ms, fbc_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, e2e_ms, attn_ms, fbc_ms = t.tolist()
+
+    flops = 4.0 * case.B * case.H * case.N * case.N * case.d  # one attention call
+    value = ws * K * flops / (ms * 1e-3) / 1e12
+    e2e_value = ws * K * flops / (e2e_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    fbc_bytes = 2 * fcase.n * 2
+    fbc_gbs = fbc_bytes / (fbc_ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": case.name, "B": case.B, "H": case.H, "N": case.N, "d": case.d,
+                   "fbc_residual": f"{fcase.rows}x{fcase.cols} bf16", "l2": "inputs larger than L2 (no flush)",
+                   "step": "dit_attn_fwd (bf16) + fbc_rel_l1"},
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": attn_tflops / peak, "traffic": None, "kernel": "attn_fwd_bf16_kernel<128>",
+                     "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                     "frac_of_spec_2250": attn_tflops / SPEC_BF16_TFLOPS},
+        "kernels": {"attn_bf16_ms": attn_ms, "attn_bf16_tflops": attn_tflops,
+                    "fbc_ms": fbc_ms, "fbc_gbs": fbc_gbs,
+                    "fbc_frac_of_measured_hbm": fbc_gbs / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if ws == 1 and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        qn = hq.view(torch.int16).numpy().view(np.uint16)
+        kn = hk.view(torch.int16).numpy().view(np.uint16)
+        vn = hv.view(torch.int16).numpy().view(np.uint16)
+        cn = hcur.view(torch.int16).numpy().view(np.uint16).reshape(fcase.rows, fcase.cols)
+        pn = hprev.view(torch.int16).numpy().view(np.uint16).reshape(fcase.rows, fcase.cols)
+        dt, fl, nr = time_oracle(case, qn, kn, vn, fcase, cn, pn, args.cpu_rows)
+        line["cpu_baseline"] = {
+            "value": fl / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{nr} query rows per head x {case.H} heads vs all {case.N} keys + residual difference "
+                      f"over the same token rows ({dt:.1f} s)", "cpu": cpu_info()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=160, help="oracle query rows per head for the cpu_baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=16, help="oracle query rows per head per reference step")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="video_long",
+                    help="video_long is the benchmark; the others serve profiling captures")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -4,9 +4,16 @@ This module only draws random numbers and encodes them as bf16 / fp32 bit
 patterns.  It holds none of the method's arithmetic and serves both the CUDA
 path (tests, bench) and the fp64 oracle, so both read identical bits.
 
-Recipe (one ``numpy.random.Generator(PCG64(seed))`` per case):
-  * draw order Q, K, V, then extras (per-channel K offsets, zeroed channels);
-  * values drawn in fp32, rounded to bf16 round-to-nearest-even on the host.
+Recipe (numpy PCG64 streams keyed by ``SeedSequence`` entropy lists, so the
+pieces can be drawn in parallel threads and still be identical every run):
+  * Q, K, V: one stream per tensor t (0, 1, 2) and head (b, h), keyed
+    [seed, t, b, h]; N(0, 1) drawn in fp32 and rounded to bf16 (round to
+    nearest even) on the host;
+  * per-channel K offsets: one stream keyed [seed, 3], N(0, std^2) per
+    (b, h, channel), added to every token of K in fp32 before the bf16
+    rounding; zeroed Q channels / token ranges are set afterwards;
+  * residual pairs: 2^24-element chunks c, r_prev from [seed, 0, c] and the
+    drift from [seed, 1, c].
 
 Workload shapes follow the token counts the pages quote: FLUX.1-dev at 1024x1024
 (4096 image + 512 text tokens, ParaAttention page, "First Block Cache"; Z-Image
@@ -16,9 +23,25 @@ vLLM-Omni "Diffusion Attention Backends"), and HunyuanVideo 720p x 129 frames
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass
 
 import numpy as np
+
+_THREADS = max(1, min(16, os.cpu_count() or 1))
+
+
+def _rng(*key: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence(list(key))))
+
+
+def _parallel(fn, items):
+    items = list(items)
+    if len(items) <= 1 or _THREADS == 1:
+        return [fn(i) for i in items]
+    with ThreadPoolExecutor(_THREADS) as ex:
+        return list(ex.map(fn, items))
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -83,20 +106,6 @@ ATTN_CASES = {c.name: c for c in (TINY, IMAGE, IMAGE_Q8, VIDEO_MID, VIDEO_LONG)}
 FBC_CASES = {c.name: c for c in (FBC_TINY, FBC_IMAGE, FBC_VIDEO_LONG)}
 
 
-def _normal_bf16(rng: np.random.Generator, shape, std: float = 1.0,
-                 chunk: int = 1 << 24) -> np.ndarray:
-    """N(0, std^2) drawn in fp32, returned as bf16 bits, chunked to bound memory."""
-    n = int(np.prod(shape))
-    out = np.empty(n, dtype=np.uint16)
-    for s in range(0, n, chunk):
-        e = min(n, s + chunk)
-        x = rng.standard_normal(e - s, dtype=np.float32)
-        if std != 1.0:
-            x *= np.float32(std)
-        out[s:e] = bf16_bits(x)
-    return out.reshape(shape)
-
-
 def attn_inputs(case: AttnCase, N: int | None = None):
     """Q, K, V as bf16 bit arrays of shape [B, H, N, d] (uint16).
 
@@ -105,18 +114,21 @@ def attn_inputs(case: AttnCase, N: int | None = None):
     """
     N = case.N if N is None else N
     shape = (case.B, case.H, N, case.d)
-    rng = np.random.Generator(np.random.PCG64(case.seed))
-    q = _normal_bf16(rng, shape)
-    k = _normal_bf16(rng, shape)
-    v = _normal_bf16(rng, shape)
+    mu = None
     if case.k_offset_std > 0.0:
-        mu = rng.standard_normal((case.B, case.H, 1, case.d), dtype=np.float32)
+        mu = _rng(case.seed, 3).standard_normal((case.B, case.H, case.d), dtype=np.float32)
         mu *= np.float32(case.k_offset_std)
-        # K = N(0,1) + mu, formed in fp32 from the bf16 draw, rounded once to bf16.
-        kb = k.reshape(case.B, case.H, N, case.d)
-        for b in range(case.B):
-            for h in range(case.H):
-                kb[b, h] = bf16_bits(bf16_to_f32(kb[b, h]) + mu[b, h])
+    out = [np.empty(shape, dtype=np.uint16) for _ in range(3)]
+
+    def fill(item):
+        t, b, h = item
+        x = _rng(case.seed, t, b, h).standard_normal((N, case.d), dtype=np.float32)
+        if t == 1 and mu is not None:
+            x += mu[b, h][None, :]
+        out[t][b, h] = bf16_bits(x)
+
+    _parallel(fill, [(t, b, h) for t in range(3) for b in range(case.B) for h in range(case.H)])
+    q, k, v = out
     if case.zero_q_channel >= 0 and case.zero_q_channel < case.d:
         q[..., case.zero_q_channel] = 0
     if case.zero_q_tokens:
@@ -125,29 +137,37 @@ def attn_inputs(case: AttnCase, N: int | None = None):
     return q, k, v
 
 
+_CHUNK = 1 << 24
+
+
 def fbc_inputs(case: FbcCase):
     """(r_cur, r_prev): r_prev ~ N(0,1), r_cur = r_prev + N(0, drift^2).
 
     fp32 cases return float32 arrays; bf16 cases return bf16 bit arrays (uint16),
-    with r_cur formed in fp32 from the bf16 r_prev and rounded once to bf16.
+    with r_prev rounded to bf16 first and r_cur formed in fp32 from that bf16
+    value plus the drift, rounded once to bf16.
     """
-    rng = np.random.Generator(np.random.PCG64(case.seed))
     n = case.n
-    if case.dtype == "f32":
-        prev = rng.standard_normal(n, dtype=np.float32)
-        drift = rng.standard_normal(n, dtype=np.float32) * np.float32(case.drift_std)
-        cur = (prev + drift).astype(np.float32)
-        return cur.reshape(case.rows, case.cols), prev.reshape(case.rows, case.cols)
-    if case.dtype == "bf16":
-        prev = _normal_bf16(rng, (n,))
-        cur = np.empty(n, dtype=np.uint16)
-        chunk = 1 << 24
-        for s in range(0, n, chunk):
-            e = min(n, s + chunk)
-            drift = rng.standard_normal(e - s, dtype=np.float32) * np.float32(case.drift_std)
-            cur[s:e] = bf16_bits(bf16_to_f32(prev[s:e]) + drift)
-        return cur.reshape(case.rows, case.cols), prev.reshape(case.rows, case.cols)
-    raise ValueError(f"unknown dtype {case.dtype}")
+    if case.dtype not in ("f32", "bf16"):
+        raise ValueError(f"unknown dtype {case.dtype}")
+    odt = np.float32 if case.dtype == "f32" else np.uint16
+    cur = np.empty(n, dtype=odt)
+    prev = np.empty(n, dtype=odt)
+
+    def fill(c):
+        s, e = c * _CHUNK, min(n, (c + 1) * _CHUNK)
+        p = _rng(case.seed, 0, c).standard_normal(e - s, dtype=np.float32)
+        drift = _rng(case.seed, 1, c).standard_normal(e - s, dtype=np.float32) * np.float32(case.drift_std)
+        if case.dtype == "f32":
+            prev[s:e] = p
+            cur[s:e] = p + drift
+        else:
+            pb = bf16_bits(p)
+            prev[s:e] = pb
+            cur[s:e] = bf16_bits(bf16_to_f32(pb) + drift)
+
+    _parallel(fill, range((n + _CHUNK - 1) // _CHUNK))
+    return cur.reshape(case.rows, case.cols), prev.reshape(case.rows, case.cols)
 
 
 def sample_rows(N: int, count: int, seed: int = 1) -> np.ndarray:
