@@ -69,14 +69,18 @@ def test_explicit_scale():
 
 
 def test_large_logits_rescaling_path():
-    # Logits grow along the key axis, so the running max moves many times:
-    # exercises the O rescale in tensor memory.
+    # Logits grow along the key axis (std up to ~15), so the running max moves
+    # by more than the rescale threshold several times: exercises the O rescale
+    # in tensor memory.  V is scaled by 1/4 (exact in bf16) so that the nearly
+    # one-hot rows keep |O| in the workloads' range, where bf16 rounding of O
+    # stays well inside the absolute bound.
     case = inputs.AttnCase("grow", 1, 2, 1024, 128, seed=9)
     q, k, v = inputs.attn_inputs(case)
     qf = inputs.bf16_to_f32(q) * np.float32(3.0)
     ramp = np.linspace(0.0, 4.0, case.N, dtype=np.float32)[None, None, :, None]
     kf = inputs.bf16_to_f32(k) * (1.0 + ramp)
     q, k = inputs.bf16_bits(qf), inputs.bf16_bits(kf)
+    v = inputs.bf16_bits(inputs.bf16_to_f32(v) * np.float32(0.25))
     assert_bf16_parity(_run(q, k, v), oracle.attention(q, k, v), "growing logits")
 
 
