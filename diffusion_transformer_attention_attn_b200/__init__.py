@@ -9,6 +9,7 @@ points raises.
 Entry points (same names as the C ABI in ``include/dit_attn.h``):
   * ``dit_attn_fwd(q, k, v, o=None, scale=None)``  — bf16 softmax attention
   * ``fbc_rel_l1(r_cur, r_prev, threshold, ...)``   — first-block-cache decision
+  * ``fbc_rel_l1_noalloc(...)``                     — the same, allocating nothing
   * ``dit_get_device_status()``                     — device-side error word
 """
 from __future__ import annotations
@@ -38,6 +39,7 @@ SIGNATURES = {
     "dit_attn_fwd": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p, _f, _p]),
     "fbc_rel_l1_workspace_bytes": (_sz, [_i64]),
     "fbc_rel_l1": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p, _sz, _p]),
+    "fbc_rel_l1_noalloc": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p]),
     "dit_get_device_status": (_i, [_p]),
     "dit_status_string": (ctypes.c_char_p, [_i]),
 }
@@ -149,6 +151,26 @@ def fbc_rel_l1(r_cur, r_prev, threshold: float, out_rel=None, out_skip=None, wor
     st = lib.fbc_rel_l1(r_cur.data_ptr(), r_prev.data_ptr(), n, dt, float(threshold), out_rel.data_ptr(),
                         out_skip.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
     _check(st, "fbc_rel_l1")
+    return out_rel, out_skip
+
+
+def fbc_rel_l1_noalloc(r_cur, r_prev, threshold: float, out_rel, out_skip, stream=None):
+    """fbc_rel_l1 without a workspace, for callers that cannot allocate device
+    memory.  The caller passes the output tensors (float64[1], int32[1]); the
+    scratch is a fixed array inside the library, shared by every call, so calls
+    must not overlap on the GPU."""
+    import torch
+    lib = load_library()
+    if r_cur.shape != r_prev.shape or r_cur.dtype != r_prev.dtype:
+        raise ValueError("r_cur and r_prev must match in shape and dtype")
+    if not (r_cur.is_contiguous() and r_prev.is_contiguous()):
+        raise ValueError("r_cur and r_prev must be contiguous")
+    dt = {torch.float32: DIT_DTYPE_F32, torch.bfloat16: DIT_DTYPE_BF16}.get(r_cur.dtype)
+    if dt is None:
+        raise TypeError("fbc_rel_l1_noalloc expects fp32 or bf16 tensors")
+    st = lib.fbc_rel_l1_noalloc(r_cur.data_ptr(), r_prev.data_ptr(), r_cur.numel(), dt, float(threshold),
+                                out_rel.data_ptr(), out_skip.data_ptr(), _stream_ptr(stream))
+    _check(st, "fbc_rel_l1_noalloc")
     return out_rel, out_skip
 
 

@@ -97,6 +97,34 @@ dit_status fbc_rel_l1(const void* r_cur, const void* r_prev, int64_t n, int dtyp
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fbc_rel_l1_noalloc — fbc_rel_l1 without a caller-provided workspace, for
+ * callers that cannot allocate device memory.  Such a caller holds only its
+ * input and output pointers: a plugin inside an inference engine, or a module
+ * in a framework whose caching allocator owns all device memory.  For it,
+ * cudaMalloc is either unavailable or an implicit device-wide synchronisation
+ * it cannot afford inside a denoising step.  No page describes this call: it is
+ * a deployment variant of fbc_rel_l1.
+ *
+ *   Arguments, result and determinism are those of fbc_rel_l1.  The call
+ *   allocates nothing.  Its scratch (a 16 B finishing ticket plus one fp64
+ *   partial pair per block, at most 1024 blocks: 16,400 B in all) is a fixed
+ *   array inside the library.  Every GPU that loads the library holds it until
+ *   the process exits.  A request whose scratch need exceeds that size returns
+ *   DIT_ERR_WORKSPACE.  With the current kernel the need is the same for every
+ *   n, so every n >= 1 fits.
+ *   The first call on each device does a one-time set-up: it looks up the
+ *   array's device address with that device current.  Make that first call
+ *   before any stream capture.
+ *   Every call clears the ticket (an asynchronous memset on `stream`) before
+ *   its launch.  All calls share one array, which keeps the last call's
+ *   partial sums, so calls that may overlap on the GPU race: calls on
+ *   different streams without ordering, or concurrent calls from several host
+ *   threads.  Order such calls, or use fbc_rel_l1 with one workspace each.
+ */
+dit_status fbc_rel_l1_noalloc(const void* r_cur, const void* r_prev, int64_t n, int dtype,
+                              float threshold, double* out_rel, int32_t* out_skip, void* stream);
+
+/*
  * dit_get_device_status — synchronises `stream`, then returns and clears the
  * device-side error word of the current device (DIT_ERR_TIMEOUT if a bounded
  * wait inside a kernel ran out since the last call), or DIT_ERR_CUDA if the
