@@ -12,6 +12,9 @@
 //   warps 4-7  softmax for Q1
 //   warp  8    TMA producer (Q once, then a ring of K and V tiles)
 //   warp  9    MMA issuer (one elected lane)
+//   warps 10-11 complete the third warpgroup (idle)
+// Registers: launched at 168 per thread; the producer warpgroup drops to 56
+// and the two softmax warpgroups rise to 224 (2·128·224 + 128·56 = 384·168).
 // Tensor memory (512 columns × 128 lanes × 32 bit):
 //   [0,128)  S0 = Q0·Kᵀ (fp32); after the softmax, P0 (bf16 pairs) in [0,64)
 //   [128,256) S1 / P1
@@ -36,7 +39,11 @@ namespace {
 
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per tile
-constexpr int kThreads = 320;     // 10 warps
+constexpr int kThreads = 384;     // 12 warps (3 warpgroups)
+constexpr int kLaunchRegs = 168;  // registers per thread the launch must provide
+constexpr int kSoftmaxRegs = 224;
+constexpr int kOtherRegs = 56;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -153,7 +160,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t smem_base = smem_u32(smem);
 
-    if (warp == kLoadWarp) {
+    if (warp >= 8) {
+      regs_dec<kOtherRegs>();
+      if (warp == kLoadWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tq);
@@ -200,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (nv[s] > 0) mbar_wait_drain(&bars.v_full[s], (nv[s] - 1) & 1);
             }
         }
-    } else if (warp == kMmaWarp) {
+      } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         const uint32_t sQ0 = smem_base + C::kQOff;
         const uint32_t sQ1 = sQ0 + C::kTileBytes;
@@ -277,8 +286,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_drain(bars.mma_done, 0);
         }
         __syncwarp();
+      }
     } else {
         // ------------------------------------------------------------ softmax (warps 0-7)
+        regs_inc<kSoftmaxRegs>();
         const int wg = warp >> 2;  // which query tile
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -312,14 +323,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (c >= valid) x[c] = -INFINITY;
                 }
             }
-            // Row max over the tile (tree of independent fmax).
+            // Row max over the tile: 8 independent chains of 3-input max.
             float mx[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx[i] = x[i];
 #pragma unroll
-            for (int c = 8; c < kBN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-            const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            for (int c = 8; c < kBN; c += 16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], x[c + i], x[c + 8 + i]);
+            const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
             const float m_new = fmaxf(m, tmax * scale_log2);
             if (j == 0) {
                 m = m_new;
@@ -331,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc_fence_after();
                     const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
+                    const float2 alpha2 = make_float2(alpha, alpha);
                     uint32_t r[32];
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
@@ -338,7 +351,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_wait_ld();
                         reg_fence32(r);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        for (int i = 0; i < 32; i += 2) {
+                            const float2 v = __fmul2_rn(
+                                make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), alpha2);
+                            r[i] = __float_as_uint(v.x);
+                            r[i + 1] = __float_as_uint(v.y);
+                        }
                         tmem_st32(tO + c * 32, r);
                     }
                     tmem_wait_st();
@@ -348,21 +366,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            const float negm = -m;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            // P = 2^(s·scale·log2e − m): packed FFMA, MUFU ex2, packed row sum.
+            const float2 c2 = make_float2(scale_log2, scale_log2);
+            const float2 negm2 = make_float2(-m, -m);
+            float2 ls[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t p[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float a = ex2_approx(fmaf(x[c * 64 + 2 * i], scale_log2, negm));
-                    const float bb = ex2_approx(fmaf(x[c * 64 + 2 * i + 1], scale_log2, negm));
-                    ls[i & 3] += a + bb;
-                    p[i] = pack_bf16x2(a, bb);
+                    const float2 t = __ffma2_rn(make_float2(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]), c2, negm2);
+                    const float2 e = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                    ls[i & 3] = __fadd2_rn(ls[i & 3], e);
+                    p[i] = pack_bf16x2(e.x, e.y);
                 }
                 tmem_st32(tS + c * 32, p);
             }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            const float2 lsum = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
+            l += lsum.x + lsum.y;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars.p_full[wg]);
@@ -407,7 +430,12 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
                      int64_t sh, int64_t sn, int B, int H, int N, float scale_log2, int* err, cudaStream_t stream) {
     using C = Cfg<D>;
     static_assert(C::kSmemBytes <= 232448, "shared memory budget");
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    // The register split inside the kernel needs the full launch allotment.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_bf16_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int n_qt = (N + kBM - 1) / kBM;
