@@ -8,6 +8,8 @@ points raises.
 
 Entry points (same names as the C ABI in ``include/dit_attn.h``):
   * ``dit_attn_fwd(q, k, v, o=None, scale=None)``  — bf16 softmax attention
+  * ``dit_attn_fwd_q8(q, k, v, ...)``              — 8-bit attention (INT8 QKᵀ, FP8 or bf16 PV)
+  * ``dit_attn_q8_quantize(q, k, v, ...)``         — its pre-pass alone
   * ``fbc_rel_l1(r_cur, r_prev, threshold, ...)``   — first-block-cache decision
   * ``fbc_rel_l1_noalloc(...)``                     — the same, allocating nothing
   * ``dit_get_device_status()``                     — device-side error word
@@ -28,6 +30,9 @@ DIT_ERR_CUDA = 4
 DIT_ERR_TIMEOUT = 5
 DIT_DTYPE_F32 = 0
 DIT_DTYPE_BF16 = 1
+DIT_PV_FP8_E4M3 = 0
+DIT_PV_BF16 = 1
+PV_MODES = {"fp8": DIT_PV_FP8_E4M3, "bf16": DIT_PV_BF16}
 
 # Every symbol include/dit_attn.h declares, with (restype, argtypes).
 _p = ctypes.c_void_p
@@ -37,6 +42,10 @@ _f = ctypes.c_float
 _sz = ctypes.c_size_t
 SIGNATURES = {
     "dit_attn_fwd": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p, _f, _p]),
+    "dit_attn_q8_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "dit_attn_fwd_q8": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p, _f, _i, _i, _p, _sz, _p]),
+    "dit_attn_q8_quantize": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _i, _i, _p, _sz, _p]),
+    "dit_attn_q8_workspace_layout": (_i, [_i, _i, _i, _i, _i, _p]),
     "fbc_rel_l1_workspace_bytes": (_sz, [_i64]),
     "fbc_rel_l1": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p, _sz, _p]),
     "fbc_rel_l1_noalloc": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p]),
@@ -112,6 +121,98 @@ def dit_attn_fwd(q, k, v, o=None, scale: float | None = None, stream=None):
                           _attn_strides(q), float(scale) if scale else 0.0, _stream_ptr(stream))
     _check(st, "dit_attn_fwd")
     return o
+
+
+def _pv(pv_mode):
+    return PV_MODES[pv_mode] if isinstance(pv_mode, str) else int(pv_mode)
+
+
+def dit_attn_q8_workspace_bytes(B: int, H: int, N: int, d: int, pv_mode="fp8") -> int:
+    return int(load_library().dit_attn_q8_workspace_bytes(B, H, N, d, _pv(pv_mode)))
+
+
+def q8_workspace(B: int, H: int, N: int, d: int, pv_mode="fp8", device=None):
+    """An (uninitialised) workspace tensor for the 8-bit path."""
+    import torch
+    n = dit_attn_q8_workspace_bytes(B, H, N, d, pv_mode)
+    if n == 0:
+        raise ValueError("unsupported shape for the 8-bit path")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+Q8_SEGMENTS = ("q_codes", "k_codes", "v_codes", "q_scale", "k_scale", "k_mean", "v_scale", "v_inv")
+
+
+def dit_attn_q8_workspace_layout(B: int, H: int, N: int, d: int, pv_mode="fp8") -> dict:
+    off = (ctypes.c_size_t * 8)()
+    _check(load_library().dit_attn_q8_workspace_layout(B, H, N, d, _pv(pv_mode), off), "dit_attn_q8_workspace_layout")
+    return dict(zip(Q8_SEGMENTS, (int(x) for x in off)))
+
+
+def q8_views(workspace, B: int, H: int, N: int, d: int, pv_mode="fp8") -> dict:
+    """Typed views of the pre-pass products inside a workspace tensor."""
+    import torch
+    off = dit_attn_q8_workspace_layout(B, H, N, d, pv_mode)
+    n_q, n_k, e = (N + 127) // 128, (N + 63) // 64, B * H * N * d
+
+    def seg(name, count, dtype, shape):
+        nbytes = count * torch.empty((), dtype=dtype).element_size()
+        return workspace[off[name]:off[name] + nbytes].view(dtype).view(shape)
+
+    views = {
+        "q_codes": seg("q_codes", e, torch.int8, (B, H, N, d)),
+        "k_codes": seg("k_codes", e, torch.int8, (B, H, N, d)),
+        "q_scale": seg("q_scale", B * H * n_q, torch.float32, (B, H, n_q)),
+        "k_scale": seg("k_scale", B * H * n_k, torch.float32, (B, H, n_k)),
+        "k_mean": seg("k_mean", B * H * d, torch.float32, (B, H, d)),
+    }
+    if _pv(pv_mode) == DIT_PV_FP8_E4M3:
+        views["v_codes"] = seg("v_codes", e, torch.uint8, (B, H, N, d))
+        views["v_scale"] = seg("v_scale", B * H * d, torch.float32, (B, H, d))
+    return views
+
+
+def _check_attn_tensors(q, k, v, o):
+    import torch
+    for t in (q, k, v) + ((o,) if o is not None else ()):
+        if t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError("expected bf16 CUDA tensors")
+        if t.shape != q.shape or t.stride() != q.stride():
+            raise ValueError("q, k, v, o must share shape and strides")
+
+
+def dit_attn_fwd_q8(q, k, v, o=None, scale: float | None = None, smooth_k: bool = True, pv_mode="fp8",
+                    workspace=None, stream=None):
+    """8-bit attention: INT8 Q (per 128 tokens) and K (per 64 tokens, optional
+    channel-mean smoothing), S in int32, P·V in FP8 e4m3 or bf16.  bf16 CUDA
+    tensors [B, H, N, 128].  Returns o."""
+    import torch
+    lib = load_library()
+    if o is None:
+        o = torch.empty_like(q)
+    _check_attn_tensors(q, k, v, o)
+    B, H, N, d = q.shape
+    if workspace is None:
+        workspace = q8_workspace(B, H, N, d, pv_mode, q.device)
+    st = lib.dit_attn_fwd_q8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), B, H, N, d, _attn_strides(q),
+                             float(scale) if scale else 0.0, int(bool(smooth_k)), _pv(pv_mode),
+                             workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(st, "dit_attn_fwd_q8")
+    return o
+
+
+def dit_attn_q8_quantize(q, k, v, smooth_k: bool = True, pv_mode="fp8", workspace=None, stream=None):
+    """Run only the 8-bit pre-pass; returns the workspace tensor."""
+    lib = load_library()
+    _check_attn_tensors(q, k, v, None)
+    B, H, N, d = q.shape
+    if workspace is None:
+        workspace = q8_workspace(B, H, N, d, pv_mode, q.device)
+    st = lib.dit_attn_q8_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, _attn_strides(q),
+                                  int(bool(smooth_k)), _pv(pv_mode), workspace.data_ptr(), workspace.numel(),
+                                  _stream_ptr(stream))
+    _check(st, "dit_attn_q8_quantize")
+    return workspace
 
 
 def fbc_rel_l1_workspace_bytes(n: int) -> int:

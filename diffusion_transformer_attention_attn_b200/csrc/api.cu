@@ -1,7 +1,7 @@
 // C ABI of libditattn.so (declared in include/dit_attn.h): argument
 // validation, TMA tensor-map encoding and launches.  Host code only; the
-// arithmetic of every call runs in the kernels of attn_bf16.cu and
-// fbc_rel_l1.cu.
+// arithmetic of every call runs in the kernels of attn_bf16.cu, attn_q8.cu,
+// q8_prepass.cu and fbc_rel_l1.cu.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -86,11 +86,12 @@ bool overlaps(const void* a, const void* b, int64_t span) {
 }
 
 // Validation shared by the attention calls.  On success fills the strides.
+// `o` may be null only when the call writes no output (need_o false).
 dit_status check_attn_args(const void* q, const void* k, const void* v, const void* o, int B, int H, int N, int d,
-                           const int64_t* strides, int64_t* sb, int64_t* sh, int64_t* sn) {
-    if (!q || !k || !v || !o) return DIT_ERR_INVALID_ARG;
+                           const int64_t* strides, int64_t* sb, int64_t* sh, int64_t* sn, bool need_o = true) {
+    if (!q || !k || !v || (need_o && !o)) return DIT_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || N < 1 || d < 1) return DIT_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DIT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (o && !aligned16(o))) return DIT_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return DIT_ERR_UNSUPPORTED;
     if (N > (1 << 30) || static_cast<int64_t>(B) * H > (1 << 24)) return DIT_ERR_UNSUPPORTED;
     if (strides) {
@@ -110,7 +111,7 @@ dit_status check_attn_args(const void* q, const void* k, const void* v, const vo
     if (*sn < d) return DIT_ERR_INVALID_ARG;
     // Extent of one tensor in bytes (for the overlap check on o).
     const int64_t span = ((B - 1) * *sb + (H - 1) * *sh + (N - 1) * *sn + d) * 2;
-    if (overlaps(o, q, span) || overlaps(o, k, span) || overlaps(o, v, span)) return DIT_ERR_INVALID_ARG;
+    if (o && (overlaps(o, q, span) || overlaps(o, k, span) || overlaps(o, v, span))) return DIT_ERR_INVALID_ARG;
     return DIT_OK;
 }
 
@@ -132,6 +133,31 @@ dit_status encode_bf16_map(CUtensorMap* map, const void* base, int B, int H, int
 }
 
 float default_scale(int d) { return 1.0f / std::sqrt(static_cast<float>(d)); }
+
+// 4-D map {128 B, N, H, B} over contiguous 8-bit codes [B, H, N, 128] inside
+// the workspace, box {128, 128, 1, 1}, 128-B swizzle.
+dit_status encode_u8_map(CUtensorMap* map, const void* base, int B, int H, int N) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return DIT_ERR_CUDA;
+    const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(N) * 128, static_cast<cuuint64_t>(H) * N * 128};
+    const cuuint32_t box[4] = {128, 128, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_INVALID_ARG;
+}
+
+// Validation shared by the 8-bit calls (after check_attn_args).
+dit_status check_q8_args(int d, int smooth_k, int pv_mode, const void* ws, size_t ws_bytes, int B, int H, int N) {
+    if (d != 128) return DIT_ERR_UNSUPPORTED;
+    if (smooth_k != 0 && smooth_k != 1) return DIT_ERR_INVALID_ARG;
+    if (pv_mode != DIT_PV_FP8_E4M3 && pv_mode != DIT_PV_BF16) return DIT_ERR_INVALID_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DIT_ERR_WORKSPACE;
+    if (ws_bytes < q8_layout(B, H, N, d, pv_mode == DIT_PV_FP8_E4M3).total) return DIT_ERR_WORKSPACE;
+    return DIT_OK;
+}
 
 }  // namespace
 }  // namespace ditk
@@ -156,6 +182,73 @@ dit_status dit_attn_fwd(const void* q, const void* k, const void* v, void* o, in
     const float scale_log2 = static_cast<float>(static_cast<double>(s) * 1.4426950408889634);
     cudaError_t e = launch_attn_bf16(tq, tk, tv, o, sb, sh, sn, B, H, N, d, scale_log2, ds->err_word,
                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+size_t dit_attn_q8_workspace_bytes(int B, int H, int N, int d, int pv_mode) {
+    if (B < 1 || H < 1 || N < 1 || d != 128) return 0;
+    if (pv_mode != DIT_PV_FP8_E4M3 && pv_mode != DIT_PV_BF16) return 0;
+    return q8_layout(B, H, N, d, pv_mode == DIT_PV_FP8_E4M3).total;
+}
+
+dit_status dit_attn_q8_workspace_layout(int B, int H, int N, int d, int pv_mode, size_t* offsets) {
+    if (!offsets || B < 1 || H < 1 || N < 1) return DIT_ERR_INVALID_ARG;
+    if (d != 128) return DIT_ERR_UNSUPPORTED;
+    if (pv_mode != DIT_PV_FP8_E4M3 && pv_mode != DIT_PV_BF16) return DIT_ERR_INVALID_ARG;
+    const Q8Layout L = q8_layout(B, H, N, d, pv_mode == DIT_PV_FP8_E4M3);
+    const size_t o[8] = {L.q_codes, L.k_codes, L.v_codes, L.q_scale, L.k_scale, L.k_mean, L.v_scale, L.v_inv};
+    for (int i = 0; i < 8; ++i) offsets[i] = o[i];
+    return DIT_OK;
+}
+
+dit_status dit_attn_q8_quantize(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                                const int64_t* strides, int smooth_k, int pv_mode, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    int64_t sb, sh, sn;
+    dit_status st = check_attn_args(q, k, v, nullptr, B, H, N, d, strides, &sb, &sh, &sn, false);
+    if (st != DIT_OK) return st;
+    if ((st = check_q8_args(d, smooth_k, pv_mode, workspace, workspace_bytes, B, H, N)) != DIT_OK) return st;
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    cudaError_t e = launch_q8_prepass(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_mode == DIT_PV_FP8_E4M3,
+                                      static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+dit_status dit_attn_fwd_q8(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                           const int64_t* strides, float scale, int smooth_k, int pv_mode, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    int64_t sb, sh, sn;
+    dit_status st = check_attn_args(q, k, v, o, B, H, N, d, strides, &sb, &sh, &sn);
+    if (st != DIT_OK) return st;
+    if (!(scale == scale) || std::isinf(scale)) return DIT_ERR_INVALID_ARG;
+    if ((st = check_q8_args(d, smooth_k, pv_mode, workspace, workspace_bytes, B, H, N)) != DIT_OK) return st;
+    const int pv_fp8 = pv_mode == DIT_PV_FP8_E4M3;
+    const Q8Layout L = q8_layout(B, H, N, d, pv_fp8);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    // The workspace must not overlap the inputs or the output.
+    const int64_t span = ((B - 1) * sb + (H - 1) * sh + (N - 1) * sn + d) * 2;
+    const int64_t wsz = static_cast<int64_t>(L.total);
+    for (const void* t : {q, k, v, static_cast<const void*>(o)}) {
+        const uintptr_t x = reinterpret_cast<uintptr_t>(t), y = reinterpret_cast<uintptr_t>(ws);
+        if (x < y + wsz && y < x + span) return DIT_ERR_WORKSPACE;
+    }
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    CUtensorMap tq8, tk8, tv;
+    if ((st = encode_u8_map(&tq8, ws + L.q_codes, B, H, N)) != DIT_OK) return st;
+    if ((st = encode_u8_map(&tk8, ws + L.k_codes, B, H, N)) != DIT_OK) return st;
+    if (pv_fp8)
+        st = encode_u8_map(&tv, ws + L.v_codes, B, H, N);
+    else
+        st = encode_bf16_map(&tv, v, B, H, N, d, sb, sh, sn);
+    if (st != DIT_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_q8_prepass(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, s);
+    if (e != cudaSuccess) return DIT_ERR_CUDA;
+    const float sc = scale > 0.f ? scale : default_scale(d);
+    const float scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
+    e = launch_attn_q8(tq8, tk8, tv, pv_fp8, ws, L, o, sb, sh, sn, B, H, N, scale_log2, ds->err_word, s);
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 

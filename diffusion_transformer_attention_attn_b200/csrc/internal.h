@@ -14,6 +14,31 @@ cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const
                              int64_t sb, int64_t sh, int64_t sn, int B, int H, int N, int d, float scale_log2,
                              int* err, cudaStream_t stream);
 
+// ---- 8-bit path (d = 128) ----------------------------------------------
+// Tokens per statistics chunk of the pre-pass.
+constexpr int kQ8StatChunk = 256;
+
+// Byte offsets of the pre-pass products inside the caller's workspace (each
+// 256-byte aligned).  Codes are [B, H, N, d] contiguous; q_scale is
+// [B, H, ceil(N/128)], k_scale [B, H, ceil(N/64)], k_mean / v_scale / v_inv
+// [B, H, d]; psum / pmax are the statistics partials [B, H, n_chunks, d].
+struct Q8Layout {
+    size_t q_codes, k_codes, v_codes, q_scale, k_scale, k_mean, v_scale, v_inv, psum, pmax, total;
+    int n_chunks;
+};
+Q8Layout q8_layout(int B, int H, int N, int d, int pv_fp8);
+
+// Statistics and quantisation of Q, K (and V when pv_fp8) into `ws`.
+cudaError_t launch_q8_prepass(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
+                              int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream);
+
+// 8-bit attention over the pre-pass products.  tq8/tk8: 4-D maps over the
+// INT8 codes {d, N, H, B}, box {128, 128, 1, 1}; tv: e4m3 codes (same box,
+// pv_fp8) or the caller's bf16 V (box {64, 128, 1, 1}).
+cudaError_t launch_attn_q8(const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv, int pv_fp8,
+                           const uint8_t* ws, const Q8Layout& L, void* o, int64_t sb, int64_t sh, int64_t sn, int B,
+                           int H, int N, float scale_log2, int* err, cudaStream_t stream);
+
 // First-block-cache residual difference (see fbc_rel_l1 in dit_attn.h).
 size_t fbc_workspace_bytes(int64_t n);
 cudaError_t launch_fbc_rel_l1(const void* cur, const void* prev, int64_t n, int dtype, float threshold,

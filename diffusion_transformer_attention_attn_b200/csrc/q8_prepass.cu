@@ -1,0 +1,280 @@
+// Pre-pass of the 8-bit attention path: statistics and quantisation of Q, K, V.
+//
+// What is computed ("TMAP image-to-video inference acceleration", section on
+// optimising operator details: 8-bit SageAttention-style attention, per-block
+// quantisation, and the zero-channel fix that guards the division by a
+// quantisation scale of zero):
+//   * Q: INT8 per block of 128 tokens (all d channels): amax over the block's
+//     valid tokens, inv = 127/amax and scale = amax/127 (fp32 divisions),
+//     code = round-half-even(x·inv) saturated to ±127.  amax = 0 gives
+//     scale = inv = 0 and all-zero codes (no NaN).
+//   * K: optionally minus its per-channel mean over all N tokens (this shifts
+//     every logit of a query row by the same amount, so softmax is unchanged),
+//     then INT8 per block of 64 tokens as above.
+//   * V (FP8 PV only): per channel, amax over all N tokens, scale = amax/448,
+//     code = e4m3(x·448/amax), round to nearest even, saturating; same guard.
+//
+// Three launches, each HBM-bound with 16-byte vector loads:
+//   q8_stats_kernel     per (b,h) and chunk of 256 tokens: fp64 column sums of
+//                       K and column |V| maxima -> partials
+//   q8_finalize_kernel  per (b,h): fixed-order fp64 sum of the partials -> the
+//                       K mean (fp64 / N, rounded once to fp32), V scales
+//   q8_quant_*_kernel   per block: amax, scale, codes
+// The K column sums are exact in fp64 for bf16 inputs of the workloads'
+// range, so the mean does not depend on the summation order.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+
+namespace ditk {
+namespace {
+
+constexpr int kStatThreads = 256;
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ const uint4* row_ptr(const void* base, int64_t sb, int64_t sh, int64_t sn, int b, int h,
+                                                int64_t n) {
+    return reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + b * sb + h * sh + n * sn);
+}
+
+// grid (n_chunks, B*H).  Thread t: 8 channels [8·(t%16), +8), rows t/16 + 16·i.
+__global__ void __launch_bounds__(kStatThreads)
+    q8_stats_kernel(const void* __restrict__ k, const void* __restrict__ v, int64_t sb, int64_t sh, int64_t sn, int H,
+                    int N, int chunk, int want_sum, int want_vmax, double* __restrict__ psum,
+                    float* __restrict__ pmax) {
+    constexpr int D = 128;
+    __shared__ double s_sum[kStatThreads / 16][D];
+    __shared__ float s_max[kStatThreads / 16][D];
+    const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int cg = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * chunk;
+    const int64_t n1 = min(static_cast<int64_t>(N), n0 + chunk);
+    double acc[8];
+    float vmax[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        acc[i] = 0.0;
+        vmax[i] = 0.f;
+    }
+    for (int64_t n = n0 + r0; n < n1; n += kStatThreads / 16) {
+        float f[8];
+        if (want_sum) {
+            unpack8(__ldg(row_ptr(k, sb, sh, sn, b, h, n) + cg), f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] += static_cast<double>(f[i]);
+        }
+        if (want_vmax) {
+            unpack8(__ldg(row_ptr(v, sb, sh, sn, b, h, n) + cg), f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) vmax[i] = fmaxf(vmax[i], fabsf(f[i]));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        s_sum[r0][cg * 8 + i] = acc[i];
+        s_max[r0][cg * 8 + i] = vmax[i];
+    }
+    __syncthreads();
+    if (threadIdx.x < D) {
+        const int c = threadIdx.x;
+        double s = 0.0;
+        float m = 0.f;
+        for (int r = 0; r < kStatThreads / 16; ++r) {
+            s += s_sum[r][c];
+            m = fmaxf(m, s_max[r][c]);
+        }
+        const int64_t idx = (static_cast<int64_t>(bh) * gridDim.x + blockIdx.x) * D + c;
+        psum[idx] = s;
+        pmax[idx] = m;
+    }
+}
+
+// grid B*H, 128 threads (one per channel).
+__global__ void q8_finalize_kernel(const double* __restrict__ psum, const float* __restrict__ pmax, int n_chunks,
+                                   int N, int want_sum, int want_vmax, float* __restrict__ k_mean,
+                                   float* __restrict__ v_scale, float* __restrict__ v_inv) {
+    constexpr int D = 128;
+    const int bh = blockIdx.x, c = threadIdx.x;
+    double s = 0.0;
+    float m = 0.f;
+    for (int i = 0; i < n_chunks; ++i) {
+        const int64_t idx = (static_cast<int64_t>(bh) * n_chunks + i) * D + c;
+        if (want_sum) s += psum[idx];
+        if (want_vmax) m = fmaxf(m, pmax[idx]);
+    }
+    k_mean[bh * D + c] = want_sum ? static_cast<float>(s / static_cast<double>(N)) : 0.f;
+    if (want_vmax) {
+        float sc = 0.f, inv = 0.f;
+        if (m > 0.f) {  // zero-scale guard
+            sc = __fdiv_rn(m, 448.f);
+            inv = __fdiv_rn(448.f, m);
+        }
+        v_scale[bh * D + c] = sc;
+        v_inv[bh * D + c] = inv;
+    }
+}
+
+__device__ __forceinline__ uint32_t s8x4(float a, float b, float c, float d) {
+    int ia, ib, ic, id;
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(ia) : "f"(a));
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(ib) : "f"(b));
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(ic) : "f"(c));
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(id) : "f"(d));
+    return (static_cast<uint32_t>(ia) & 0xFFu) | ((static_cast<uint32_t>(ib) & 0xFFu) << 8) |
+           ((static_cast<uint32_t>(ic) & 0xFFu) << 16) | ((static_cast<uint32_t>(id) & 0xFFu) << 24);
+}
+
+// INT8 per block of BLK tokens.  grid (ceil(N/BLK), B*H), 256 threads:
+// thread t holds channels [8·(t%16), +8) of rows t/16 + 16·i of the block.
+template <int BLK>
+__global__ void __launch_bounds__(kQuantThreads)
+    q8_quant_int8_kernel(const void* __restrict__ x, int64_t sb, int64_t sh, int64_t sn, int H, int N,
+                         const float* __restrict__ mean, int8_t* __restrict__ codes, float* __restrict__ scales) {
+    constexpr int D = 128;
+    constexpr int kRows = BLK / 16;  // rows per thread
+    __shared__ float s_red[kQuantThreads / 32];
+    const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int cg = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * BLK;
+    float mu[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mu[i] = mean ? mean[bh * D + cg * 8 + i] : 0.f;
+    float val[kRows][8];
+    float amax = 0.f;
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+        const int64_t n = t0 + r0 + 16 * r;
+        if (n < N) {
+            unpack8(__ldg(row_ptr(x, sb, sh, sn, b, h, n) + cg), val[r]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (mean) val[r][i] = __fsub_rn(val[r][i], mu[i]);
+                amax = fmaxf(amax, fabsf(val[r][i]));
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, s_red[w]);
+    float inv = 0.f, scale = 0.f;
+    if (amax > 0.f) {  // zero-scale guard
+        inv = __fdiv_rn(127.f, amax);
+        scale = __fdiv_rn(amax, 127.f);
+    }
+    if (threadIdx.x == 0) scales[static_cast<int64_t>(bh) * gridDim.x + blockIdx.x] = scale;
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+        const int64_t n = t0 + r0 + 16 * r;
+        if (n < N) {
+            float q[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(val[r][i], inv);
+            uint2 w;
+            w.x = s8x4(q[0], q[1], q[2], q[3]);
+            w.y = s8x4(q[4], q[5], q[6], q[7]);
+            *reinterpret_cast<uint2*>(codes + (static_cast<int64_t>(bh) * N + n) * D + cg * 8) = w;
+        }
+    }
+}
+
+// Two fp32 -> packed e4m3x2 (round to nearest even, saturating); `lo` in bits 0-7.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// FP8 e4m3 per channel.  grid (ceil(N/128), B*H), 256 threads, as above.
+__global__ void __launch_bounds__(kQuantThreads)
+    q8_quant_e4m3_kernel(const void* __restrict__ x, int64_t sb, int64_t sh, int64_t sn, int H, int N,
+                         const float* __restrict__ v_inv, uint8_t* __restrict__ codes) {
+    constexpr int D = 128;
+    const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int cg = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+    float inv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) inv[i] = v_inv[bh * D + cg * 8 + i];
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * 128;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int64_t n = t0 + r0 + 16 * r;
+        if (n < N) {
+            float f[8];
+            unpack8(__ldg(row_ptr(x, sb, sh, sn, b, h, n) + cg), f);
+            uint2 w;
+            w.x = e4m3x2(__fmul_rn(f[0], inv[0]), __fmul_rn(f[1], inv[1])) |
+                  (e4m3x2(__fmul_rn(f[2], inv[2]), __fmul_rn(f[3], inv[3])) << 16);
+            w.y = e4m3x2(__fmul_rn(f[4], inv[4]), __fmul_rn(f[5], inv[5])) |
+                  (e4m3x2(__fmul_rn(f[6], inv[6]), __fmul_rn(f[7], inv[7])) << 16);
+            *reinterpret_cast<uint2*>(codes + (static_cast<int64_t>(bh) * N + n) * D + cg * 8) = w;
+        }
+    }
+}
+
+}  // namespace
+
+Q8Layout q8_layout(int B, int H, int N, int d, int pv_fp8) {
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    Q8Layout L{};
+    const size_t BH = static_cast<size_t>(B) * H;
+    const size_t elems = BH * static_cast<size_t>(N) * d;
+    L.n_chunks = (N + kQ8StatChunk - 1) / kQ8StatChunk;
+    size_t off = 0;
+    L.q_codes = off; off = up(off + elems);
+    L.k_codes = off; off = up(off + elems);
+    L.v_codes = off; off = up(off + (pv_fp8 ? elems : 0));
+    L.q_scale = off; off = up(off + BH * ((N + 127) / 128) * sizeof(float));
+    L.k_scale = off; off = up(off + BH * ((N + 63) / 64) * sizeof(float));
+    L.k_mean = off;  off = up(off + BH * d * sizeof(float));
+    L.v_scale = off; off = up(off + BH * d * sizeof(float));
+    L.v_inv = off;   off = up(off + BH * d * sizeof(float));
+    L.psum = off;    off = up(off + BH * L.n_chunks * d * sizeof(double));
+    L.pmax = off;    off = up(off + BH * L.n_chunks * d * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+cudaError_t launch_q8_prepass(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
+                              int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
+    const Q8Layout L = q8_layout(B, H, N, 128, pv_fp8);
+    const int BH = B * H;
+    double* psum = reinterpret_cast<double*>(ws + L.psum);
+    float* pmax = reinterpret_cast<float*>(ws + L.pmax);
+    float* k_mean = reinterpret_cast<float*>(ws + L.k_mean);
+    float* v_scale = reinterpret_cast<float*>(ws + L.v_scale);
+    float* v_inv = reinterpret_cast<float*>(ws + L.v_inv);
+    if (smooth_k || pv_fp8) {
+        q8_stats_kernel<<<dim3(L.n_chunks, BH), kStatThreads, 0, stream>>>(k, v, sb, sh, sn, H, N, kQ8StatChunk,
+                                                                           smooth_k, pv_fp8, psum, pmax);
+        q8_finalize_kernel<<<BH, 128, 0, stream>>>(psum, pmax, L.n_chunks, N, smooth_k, pv_fp8, k_mean, v_scale,
+                                                   v_inv);
+    }
+    q8_quant_int8_kernel<128><<<dim3((N + 127) / 128, BH), kQuantThreads, 0, stream>>>(
+        q, sb, sh, sn, H, N, nullptr, reinterpret_cast<int8_t*>(ws + L.q_codes),
+        reinterpret_cast<float*>(ws + L.q_scale));
+    q8_quant_int8_kernel<64><<<dim3((N + 63) / 64, BH), kQuantThreads, 0, stream>>>(
+        k, sb, sh, sn, H, N, smooth_k ? k_mean : nullptr, reinterpret_cast<int8_t*>(ws + L.k_codes),
+        reinterpret_cast<float*>(ws + L.k_scale));
+    if (pv_fp8)
+        q8_quant_e4m3_kernel<<<dim3((N + 127) / 128, BH), kQuantThreads, 0, stream>>>(
+            v, sb, sh, sn, H, N, v_inv, ws + L.v_codes);
+    return cudaGetLastError();
+}
+
+}  // namespace ditk

@@ -41,6 +41,9 @@ typedef enum {
 
 typedef enum { DIT_DTYPE_F32 = 0, DIT_DTYPE_BF16 = 1 } dit_dtype;
 
+/* Precision of the P·V contraction of the 8-bit path. */
+typedef enum { DIT_PV_FP8_E4M3 = 0, DIT_PV_BF16 = 1 } dit_pv_mode;
+
 /*
  * dit_attn_fwd — softmax attention O = softmax(scale · Q Kᵀ) V, per (b, h),
  * over all N keys (no mask: the text and visual tokens form one joint,
@@ -67,6 +70,59 @@ typedef enum { DIT_DTYPE_F32 = 0, DIT_DTYPE_BF16 = 1 } dit_dtype;
 dit_status dit_attn_fwd(const void* q, const void* k, const void* v, void* o,
                         int B, int H, int N, int d, const int64_t* strides,
                         float scale, void* stream);
+
+/*
+ * dit_attn_fwd_q8 — the same attention with 8-bit operands.
+ *
+ * Defined by: "TMAP image-to-video inference acceleration" (joto.ai), section
+ * on optimising operator details: 8-bit SageAttention-style attention with
+ * per-block quantisation.  An all-zero channel made the quantisation scale 0
+ * and the division by it turned the video black (NaN); the scale here is
+ * guarded.  Recipe:
+ *   Q  -> INT8 per block of 128 tokens (all d channels);
+ *   K  -> optionally minus its per-channel mean over the N tokens (smooth_k;
+ *         a per-row logit shift, so the softmax is unchanged), then INT8 per
+ *         block of 64 tokens;
+ *   INT8 scales: amax over the block's valid tokens, scale = amax/127,
+ *         codes = round-half-even(x·127/amax) in [-127, 127]; amax = 0 gives
+ *         scale 0 and zero codes;
+ *   S = Q8·K8ᵀ in int32, dequantised by q_scale·k_scale;
+ *   P·V in FP8 e4m3 (pv_mode DIT_PV_FP8_E4M3: V per channel, scale
+ *         amax/448; P scaled by 2^6.5 before e4m3) or in bf16 (DIT_PV_BF16:
+ *         P bf16, V as given).
+ *
+ *   Arguments as dit_attn_fwd, plus:
+ *   smooth_k        0 or 1.
+ *   pv_mode         a dit_pv_mode.
+ *   workspace       device memory of dit_attn_q8_workspace_bytes(...) bytes,
+ *                   256-byte aligned, not overlapping q, k, v or o; no
+ *                   initialisation needed.  It receives the codes and scales
+ *                   (layout: dit_attn_q8_workspace_layout).
+ *   d must be 128 (others: DIT_ERR_UNSUPPORTED).
+ *   Launches the pre-pass (3-5 kernels) and the attention kernel on `stream`.
+ */
+size_t dit_attn_q8_workspace_bytes(int B, int H, int N, int d, int pv_mode);
+dit_status dit_attn_fwd_q8(const void* q, const void* k, const void* v, void* o,
+                           int B, int H, int N, int d, const int64_t* strides,
+                           float scale, int smooth_k, int pv_mode,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * dit_attn_q8_quantize — only the pre-pass of dit_attn_fwd_q8: writes the
+ * codes and scales into `workspace` (arguments as dit_attn_fwd_q8, no o).
+ *
+ * dit_attn_q8_workspace_layout — byte offsets inside the workspace, in this
+ * order: Q codes (int8 [B,H,N,d]), K codes (int8 [B,H,N,d]), V codes (e4m3
+ * [B,H,N,d], FP8 mode only), Q scales (fp32 [B,H,ceil(N/128)]), K scales
+ * (fp32 [B,H,ceil(N/64)]), K channel means (fp32 [B,H,d]; zeros when
+ * smooth_k = 0), V scales (fp32 [B,H,d]), V inverse scales (fp32 [B,H,d]).
+ * offsets: host array of 8 size_t.
+ */
+dit_status dit_attn_q8_quantize(const void* q, const void* k, const void* v,
+                                int B, int H, int N, int d, const int64_t* strides,
+                                int smooth_k, int pv_mode,
+                                void* workspace, size_t workspace_bytes, void* stream);
+dit_status dit_attn_q8_workspace_layout(int B, int H, int N, int d, int pv_mode, size_t* offsets);
 
 /*
  * fbc_rel_l1 — first-block-cache residual difference and decision:

@@ -109,3 +109,47 @@ def test_product_path_does_not_reach_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "liboracle" not in text, f
+
+
+def test_q8_workspace_size_and_layout(lib):
+    assert lib.dit_attn_q8_workspace_bytes(1, 2, 256, 64, 0) == 0          # d = 64: not served
+    assert lib.dit_attn_q8_workspace_bytes(1, 2, 256, 128, 7) == 0         # bad mode
+    fp8 = lib.dit_attn_q8_workspace_bytes(1, 24, 4608, 128, dit.DIT_PV_FP8_E4M3)
+    bf = lib.dit_attn_q8_workspace_bytes(1, 24, 4608, 128, dit.DIT_PV_BF16)
+    codes = 24 * 4608 * 128
+    assert fp8 >= 3 * codes and bf >= 2 * codes and fp8 - bf >= codes
+    off = dit.dit_attn_q8_workspace_layout(1, 24, 4608, 128, "fp8")
+    vals = [off[k] for k in dit.Q8_SEGMENTS]
+    assert all(v % 256 == 0 for v in vals) and vals == sorted(vals) and vals[-1] < fp8
+    assert off["k_codes"] - off["q_codes"] >= codes
+
+
+WS = 0x50000000
+
+
+def _q8(lib, q=Q, k=K, v=V, o=O, B=1, H=2, N=256, d=128, smooth=1, mode=0, ws=WS, wsb=None):
+    if wsb is None:
+        wsb = lib.dit_attn_q8_workspace_bytes(B, H, N, 128, 0)
+    return lib.dit_attn_fwd_q8(q, k, v, o, B, H, N, d, None, 0.0, smooth, mode, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=64), dit.DIT_ERR_UNSUPPORTED),
+    (dict(mode=5), dit.DIT_ERR_INVALID_ARG),
+    (dict(smooth=2), dit.DIT_ERR_INVALID_ARG),
+    (dict(ws=0), dit.DIT_ERR_WORKSPACE),
+    (dict(ws=WS + 128), dit.DIT_ERR_WORKSPACE),                 # not 256-byte aligned
+    (dict(wsb=1024), dit.DIT_ERR_WORKSPACE),
+    (dict(ws=Q), dit.DIT_ERR_WORKSPACE),                        # overlaps q
+    (dict(v=0), dit.DIT_ERR_INVALID_ARG),
+    (dict(N=0), dit.DIT_ERR_INVALID_ARG),
+])
+def test_q8_argument_errors(lib, kw, status):
+    assert _q8(lib, **kw) == status
+
+
+def test_q8_quantize_argument_errors(lib):
+    wsb = lib.dit_attn_q8_workspace_bytes(1, 2, 256, 128, 0)
+    assert lib.dit_attn_q8_quantize(Q, K, V, 1, 2, 256, 64, None, 1, 0, WS, wsb, None) == dit.DIT_ERR_UNSUPPORTED
+    assert lib.dit_attn_q8_quantize(Q, K, V, 1, 2, 256, 128, None, 1, 0, WS, 100, None) == dit.DIT_ERR_WORKSPACE
+    assert lib.dit_attn_q8_quantize(0, K, V, 1, 2, 256, 128, None, 1, 0, WS, wsb, None) == dit.DIT_ERR_INVALID_ARG
