@@ -5,12 +5,14 @@ One step = one pass of the whole hot path over one batch of synthetic input of
 the long-video workload (HunyuanVideo 720p x 129 frames: B=1, H=24,
 N=119056 joint tokens, d=128, bf16 Q/K/V ~ N(0,1) with K per-channel offsets
 ~ N(0, 2^2)):
-  * dit_attn_fwd  — bf16 softmax attention over all 119056 keys
-  * fbc_rel_l1    — first-block-cache decision over that model's residual pair
-                    (119056 x 3072 bf16, drift N(0, 0.03^2), threshold 0.08)
+  * dit_attn_fwd     — bf16 softmax attention over all 119056 keys
+  * dit_attn_fwd_q8  — the same attention on 8-bit operands (pre-pass: INT8
+                       Q/K with K-mean smoothing, e4m3 V; INT8 QK^T, FP8 PV)
+  * fbc_rel_l1       — first-block-cache decision over that model's residual
+                       pair (119056 x 3072 bf16, drift N(0, 0.03^2), thr 0.08)
 
-The metric is attention TFLOP/s (4*B*H*N^2*d per attention call) over the
-whole step.  Inputs (2.2 GB of Q/K/V, 1.5 GB of residuals) are far larger than
+The metric is attention TFLOP/s (4*B*H*N^2*d per attention call, two calls
+per step) over the whole step.  Inputs (2.2 GB of Q/K/V, 1.5 GB of residuals) are far larger than
 the 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -240,6 +242,7 @@ def run_ours(args):
     hq, hk, hv = (pinned_bf16(t) for t in (q, k, v))
     hcur, hprev = pinned_bf16(cur), pinned_bf16(prev)
     ho = torch.empty_like(hq).pin_memory()
+    ho8 = torch.empty_like(hq).pin_memory()
     hrel = torch.empty(1, dtype=torch.float64).pin_memory()
     hskip = torch.empty(1, dtype=torch.int32).pin_memory()
     del q, k, v, cur, prev
@@ -250,13 +253,20 @@ def run_ours(args):
     drel = torch.empty(1, dtype=torch.float64, device=dev)
     dskip = torch.empty(1, dtype=torch.int32, device=dev)
     fws = dit.fbc_workspace(dcur.numel(), dev)
+    do8 = torch.empty_like(dq)
+    qws = dit.q8_workspace(case.B, case.H, case.N, case.d, "fp8", dev)
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
 
-    launches_per_step = 2  # attention + residual difference
+    # bf16 attention 1 + 8-bit (stats, finalize, quantise Q, K, V, attention) 6 + fbc 1
+    launches_per_step = 8
+
+    def q8(o):
+        dit.dit_attn_fwd_q8(dq, dk, dv, o=o, smooth_k=True, pv_mode="fp8", workspace=qws)
 
     def step():
         dit.dit_attn_fwd(dq, dk, dv, o=do)
+        q8(do8)
         dit.fbc_rel_l1(dcur, dprev, fcase.threshold, out_rel=drel, out_skip=dskip, workspace=fws)
 
     for _ in range(args.warmup):
@@ -277,6 +287,7 @@ def run_ours(args):
     K = args.steps
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e8 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     ef = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     barrier()
     torch.cuda.synchronize(dev)
@@ -286,6 +297,9 @@ def run_ours(args):
         ea[i][0].record(stream)
         dit.dit_attn_fwd(dq, dk, dv, o=do)
         ea[i][1].record(stream)
+        e8[i][0].record(stream)
+        q8(do8)
+        e8[i][1].record(stream)
         ef[i][0].record(stream)
         dit.fbc_rel_l1(dcur, dprev, fcase.threshold, out_rel=drel, out_skip=dskip, workspace=fws)
         ef[i][1].record(stream)
@@ -295,6 +309,7 @@ def run_ours(args):
     clocks = sampler.stop()
     ms = ev[0].elapsed_time(ev[1])
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ea)
+    q8_ms = statistics.mean(a.elapsed_time(b) for a, b in e8)
     fbc_ms = statistics.mean(a.elapsed_time(b) for a, b in ef)
     st = dit.dit_get_device_status()
     if st != 0:
@@ -310,7 +325,9 @@ def run_ours(args):
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         dit.dit_attn_fwd(dq, dk, dv, o=do)
+        q8(do8)
         ho.copy_(do, non_blocking=True)
+        ho8.copy_(do8, non_blocking=True)
         dcur.copy_(hcur, non_blocking=True)
         dprev.copy_(hprev, non_blocking=True)
         dit.fbc_rel_l1(dcur, dprev, fcase.threshold, out_rel=drel, out_skip=dskip, workspace=fws)
@@ -321,41 +338,67 @@ def run_ours(args):
     barrier()
     e2e_ms = e1[0].elapsed_time(e1[1])
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcur, hprev))
-    d2h = ho.numel() * ho.element_size() + 8 + 4
+    d2h = 2 * ho.numel() * ho.element_size() + 8 + 4
+
+    # ---- the 8-bit pre-pass alone (informational, outside the timed step)
+    ep = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ep[0].record(stream)
+    for _ in range(K):
+        dit.dit_attn_q8_quantize(dq, dk, dv, smooth_k=True, pv_mode="fp8", workspace=qws)
+    ep[1].record(stream)
+    torch.cuda.synchronize(dev)
+    prepass_ms = ep[0].elapsed_time(ep[1]) / K
 
     # ---- max over ranks
-    t = torch.tensor([ms, e2e_ms, attn_ms, fbc_ms], dtype=torch.float64, device=dev)
+    t = torch.tensor([ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms], dtype=torch.float64, device=dev)
     if ws > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms, attn_ms, fbc_ms = t.tolist()
+    ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms = t.tolist()
 
     flops = 4.0 * case.B * case.H * case.N * case.N * case.d  # one attention call
-    value = ws * K * flops / (ms * 1e-3) / 1e12
-    e2e_value = ws * K * flops / (e2e_ms * 1e-3) / 1e12
+    value = ws * K * 2 * flops / (ms * 1e-3) / 1e12
+    e2e_value = ws * K * 2 * flops / (e2e_ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    q8_tflops = flops / (q8_ms * 1e-3) / 1e12
+    q8_attn_tflops = flops / ((q8_ms - prepass_ms) * 1e-3) / 1e12
+    # FP8/INT8 dense peak: the measured bf16 figure x the nominal 2x ratio
+    peak8 = 2.0 * peak
     fbc_bytes = 2 * fcase.n * 2
     fbc_gbs = fbc_bytes / (fbc_ms * 1e-3) / 1e9
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
+        "dtype": "bf16+int8/fp8", "data": "synthetic",
         "config": {"workload": case.name, "B": case.B, "H": case.H, "N": case.N, "d": case.d,
                    "fbc_residual": f"{fcase.rows}x{fcase.cols} bf16", "l2": "inputs larger than L2 (no flush)",
-                   "step": "dit_attn_fwd (bf16) + fbc_rel_l1"},
-        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": attn_tflops / peak, "traffic": None, "kernel": "attn_fwd_bf16_kernel<128>",
-                     "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
-                     "frac_of_spec_2250": attn_tflops / SPEC_BF16_TFLOPS},
+                   "step": "dit_attn_fwd (bf16) + dit_attn_fwd_q8 (smooth_k, FP8 PV) + fbc_rel_l1"},
+        "roofline": None,
         "kernels": {"attn_bf16_ms": attn_ms, "attn_bf16_tflops": attn_tflops,
+                    "q8_call_ms": q8_ms, "q8_call_tflops": q8_tflops, "q8_prepass_ms": prepass_ms,
+                    "q8_attn_tflops": q8_attn_tflops, "q8_attn_frac_of_fp8_peak": q8_attn_tflops / peak8,
+                    "q8_speedup_vs_bf16": attn_ms / q8_ms,
                     "fbc_ms": fbc_ms, "fbc_gbs": fbc_gbs,
                     "fbc_frac_of_measured_hbm": fbc_gbs / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
+    roof_bf16 = {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                 "frac": attn_tflops / peak, "traffic": None, "kernel": "attn_fwd_bf16_kernel<128>",
+                 "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                 "frac_of_spec_2250": attn_tflops / SPEC_BF16_TFLOPS}
+    roof_q8 = {"bound": "tensor", "achieved": q8_attn_tflops, "peak": peak8, "unit": "TFLOP/s",
+               "frac": q8_attn_tflops / peak8, "traffic": None, "kernel": "attn_fwd_q8_kernel<true>",
+               "peak_source": f"{peak_src} bf16 sustained x 2 (nominal FP8/INT8 : bf16 ratio)",
+               "frac_of_spec_4500": q8_attn_tflops / (2 * SPEC_BF16_TFLOPS)}
+    # the dominant kernel by time carries the roofline; the other is reported beside it
+    if attn_ms >= q8_ms - prepass_ms:
+        line["roofline"], line["roofline_other"] = roof_bf16, roof_q8
+    else:
+        line["roofline"], line["roofline_other"] = roof_q8, roof_bf16
     if ws == 1 and rank == 0 and not args.no_cpu_baseline:
         import oracle
         oracle.build()

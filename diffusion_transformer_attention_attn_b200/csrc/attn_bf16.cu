@@ -16,7 +16,8 @@
 // Registers: launched at 168 per thread; the producer warpgroup drops to 56
 // and the two softmax warpgroups rise to 224 (2·128·224 + 128·56 = 384·168).
 // Tensor memory (512 columns × 128 lanes × 32 bit):
-//   [0,128)  S0 = Q0·Kᵀ (fp32); after the softmax, P0 (bf16 pairs) in [0,64)
+//   [0,128)  S0 = Q0·Kᵀ (fp32); after the softmax, P0 (bf16 pairs) in [0,64),
+//            written and published in two 64-key halves
 //   [128,256) S1 / P1
 //   [256,256+d) O0 accumulator;  [256+d, 256+2d) O1 accumulator
 // The MMA warp alternates the two tiles so that the tensor core computes
@@ -31,6 +32,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
@@ -43,6 +46,11 @@ constexpr int kThreads = 384;     // 12 warps (3 warpgroups)
 constexpr int kLaunchRegs = 168;  // registers per thread the launch must provide
 constexpr int kSoftmaxRegs = 224;
 constexpr int kOtherRegs = 56;
+// Pairs of exponentials (out of every 8) evaluated on the FMA pipe.
+constexpr int kEmuOf8 = 1;
+// Publish P in two 64-key halves (the MMA warp starts P·V on the first half
+// while the second is computed) or whole.
+constexpr bool kSplitP = false;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -59,8 +67,8 @@ struct Cfg {
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
-    //           s_full[2], p_full[2], o_ready[2], mma_done
-    static constexpr int kNumBars = 1 + 4 * kStages + 6 + 1;
+    //           s_full[2], p_full[2 tiles × 2 halves], o_ready[2], mma_done
+    static constexpr int kNumBars = 1 + 4 * kStages + 8 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;    // + slack for 1024-B alignment
     // S tiles: M=128 rows, N=128 keys, K-major A (Q) and B (K).
@@ -93,23 +101,18 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
     r.v_empty = r.v_full + C::kStages;
     r.s_full = r.v_empty + C::kStages;
     r.p_full = r.s_full + 2;
-    r.o_ready = r.p_full + 2;
+    r.o_ready = r.p_full + 4;
     r.mma_done = r.o_ready + 2;
     return r;
 }
 
-// K-major operand (Q or K tile) for k-step kk (16 bf16 along d): the d-halves
-// are separate 16 KB swizzle panels; inside a panel, +32 B per k-step.
-template <int D>
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_saddr, int kk) {
-    const uint32_t a = tile_saddr + (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    return smem_desc_sw128(a, 16, 1024);
-}
-// MN-major V tile for key-step kk (16 keys): +16 rows × 128 B per step;
-// LBO = distance between the 64-wide d panels, SBO = 8 keys × 128 B.
-__device__ __forceinline__ uint64_t desc_v(uint32_t tile_saddr, int kk) {
-    return smem_desc_sw128(tile_saddr + kk * 16 * 128, kHalfBytes, 1024);
-}
+// K-major operand (Q or K tile, 128-B swizzle, SBO = 8 rows × 128 B) at
+// k-step kk (16 bf16 along d): the d-halves are separate 16 KB panels;
+// inside a panel, +32 B per k-step.
+__host__ __device__ constexpr uint32_t kmajor_off(int kk) { return (kk >> 2) * kHalfBytes + (kk & 3) * 32; }
+// MN-major V tile (LBO = distance between the 64-wide d panels, SBO = 8 keys ×
+// 128 B) at key-step kk (16 keys): +16 rows × 128 B.
+__host__ __device__ constexpr uint32_t v_off(int kk) { return kk * 16 * 128; }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -143,7 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars.s_full[t], 1);
-            mbar_init(&bars.p_full[t], kBM);
+            mbar_init(&bars.p_full[2 * t], kBM);
+            mbar_init(&bars.p_full[2 * t + 1], kBM);
             mbar_init(&bars.o_ready[t], 1);
         }
         mbar_init(bars.mma_done, 1);
@@ -211,68 +215,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        const uint32_t sQ0 = smem_base + C::kQOff;
-        const uint32_t sQ1 = sQ0 + C::kTileBytes;
+        const SDesc dQ0 = sdesc_sw128(smem_base + C::kQOff, 16, 1024);
+        const SDesc dQ1 = sdesc_add(dQ0, C::kTileBytes);
+        const SDesc dK0 = sdesc_sw128(smem_base + C::kKOff, 16, 1024);
+        const SDesc dV0 = sdesc_sw128(smem_base + C::kVOff, kHalfBytes, 1024);
         const uint32_t tS0 = tmem, tS1 = tmem + 128;
         const uint32_t tO0 = tmem + 256, tO1 = tmem + 256 + D;
+        auto issue_s = [&](uint32_t tS, SDesc dQ, SDesc dK) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_ss<0>(tS, sdesc_add(dQ, kmajor_off(kk)), sdesc_add(dK, kmajor_off(kk)), C::kIdescQK, kk > 0);
+        };
         bool ok = mbar_wait(bars.q_full, 0, abort_flag, err) && mbar_wait(&bars.k_full[0], 0, abort_flag, err);
         if (ok) {
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t sK = smem_base + C::kKOff;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_bf16_ss(tS0, desc_kmajor<D>(sQ0, kk), desc_kmajor<D>(sK, kk), C::kIdescQK, kk > 0);
+                issue_s(tS0, dQ0, dK0);
                 mma_commit(&bars.s_full[0]);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_bf16_ss(tS1, desc_kmajor<D>(sQ1, kk), desc_kmajor<D>(sK, kk), C::kIdescQK, kk > 0);
+                issue_s(tS1, dQ1, dK0);
                 mma_commit(&bars.s_full[1]);
                 mma_commit(&bars.k_empty[0]);
             }
             __syncwarp();
             for (int j = 0; j < nkv && ok; ++j) {
                 const int vs = j % C::kStages;
-                const uint32_t sV = smem_base + C::kVOff + vs * C::kTileBytes;
+                const SDesc dV = sdesc_add(dV0, vs * C::kTileBytes);
                 const bool more = j + 1 < nkv;
                 const int ks = (j + 1) % C::kStages;
-                const uint32_t sK = smem_base + C::kKOff + ks * C::kTileBytes;
-                ok = mbar_wait(&bars.v_full[vs], (j / C::kStages) & 1, abort_flag, err) &&
-                     mbar_wait(&bars.p_full[0], j & 1, abort_flag, err);
+                const SDesc dK = sdesc_add(dK0, ks * C::kTileBytes);
+                ok = mbar_wait(&bars.v_full[vs], (j / C::kStages) & 1, abort_flag, err);
                 if (!ok) break;
-                tc_fence_after();
-                if (lane == 0) {
+                // O_t += P_t·V (in two 64-key halves when P is published in halves).
+                auto issue_pv = [&](int t, uint32_t tO, uint32_t tP) {
+                    constexpr int kParts = kSplitP ? 2 : 1;
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        mma_bf16_ts(tO0, tS0 + kk * 8, desc_v(sV, kk), C::kIdescPV, (j > 0 || kk > 0));
-                    mma_commit(&bars.o_ready[0]);
-                }
+                    for (int hf = 0; hf < kParts; ++hf) {
+                        ok = ok && mbar_wait(&bars.p_full[2 * t + hf], j & 1, abort_flag, err);
+                        if (!ok) return;
+                        tc_fence_after();
+                        if (lane == 0) {
+#pragma unroll
+                            for (int kk = hf * (8 / kParts); kk < (hf + 1) * (8 / kParts); ++kk)
+                                mma_ts<0>(tO, tP + kk * 8, sdesc_add(dV, v_off(kk)), C::kIdescPV, (j > 0 || kk > 0));
+                        }
+                        __syncwarp();
+                    }
+                };
+                issue_pv(0, tO0, tS0);
+                if (!ok) break;
+                if (lane == 0) mma_commit(&bars.o_ready[0]);
                 __syncwarp();
                 if (more) {
                     ok = mbar_wait(&bars.k_full[ks], ((j + 1) / C::kStages) & 1, abort_flag, err);
                     if (!ok) break;
                     tc_fence_after();
                     if (lane == 0) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            mma_bf16_ss(tS0, desc_kmajor<D>(sQ0, kk), desc_kmajor<D>(sK, kk), C::kIdescQK, kk > 0);
+                        issue_s(tS0, dQ0, dK);
                         mma_commit(&bars.s_full[0]);
                     }
                     __syncwarp();
                 }
-                ok = mbar_wait(&bars.p_full[1], j & 1, abort_flag, err);
+                issue_pv(1, tO1, tS1);
                 if (!ok) break;
-                tc_fence_after();
                 if (lane == 0) {
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        mma_bf16_ts(tO1, tS1 + kk * 8, desc_v(sV, kk), C::kIdescPV, (j > 0 || kk > 0));
                     mma_commit(&bars.o_ready[1]);
                     mma_commit(&bars.v_empty[vs]);
                     if (more) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            mma_bf16_ss(tS1, desc_kmajor<D>(sQ1, kk), desc_kmajor<D>(sK, kk), C::kIdescQK, kk > 0);
+                        issue_s(tS1, dQ1, dK);
                         mma_commit(&bars.s_full[1]);
                         mma_commit(&bars.k_empty[ks]);
                     }
@@ -302,36 +311,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = mbar_wait(&bars.s_full[wg], j & 1, abort_flag, err);
             if (!ok) break;
             tc_fence_after();
-            float x[kBN];
-            {
-                uint32_t r[kBN / 32][32];
+            uint32_t r[kBN / 32][32];
+            auto X = [&](int col) { return __uint_as_float(r[col >> 5][col & 31]); };
+            const int valid = N - j * kBN;  // keys of this tile below N
+            // Row max over the tile; keys past N are left out.  Full tiles load
+            // S in 32-column chunks and fold each chunk into 8 independent
+            // 3-input max chains while the next chunk is in flight.
+            float tmax;
+            if (valid >= kBN) {
+                float mx[8];
+                tmem_ld32(tS, r[0]);
+                tmem_wait_ld();
+                reg_fence32(r[0]);
+#pragma unroll
+                for (int c = 0; c < kBN / 32; ++c) {
+                    if (c + 1 < kBN / 32) tmem_ld32(tS + (c + 1) * 32, r[c + 1]);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float a = X(c * 32 + i), b2 = X(c * 32 + 8 + i), c3 = X(c * 32 + 16 + i),
+                                    d4 = X(c * 32 + 24 + i);
+                        mx[i] = c == 0 ? fmax3(a, b2, fmaxf(c3, d4)) : fmax3(mx[i], fmax3(a, b2, c3), d4);
+                    }
+                    if (c + 1 < kBN / 32) {
+                        tmem_wait_ld();
+                        reg_fence32(r[c + 1]);
+                    }
+                }
+                tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+            } else {
 #pragma unroll
                 for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, r[c]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < kBN / 32; ++c) {
-                    reg_fence32(r[c]);
+                for (int c = 0; c < kBN / 32; ++c) reg_fence32(r[c]);
+                tmax = -INFINITY;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[c][i]);
-                }
+                for (int c = 0; c < kBN; ++c)
+                    if (c < valid) tmax = fmaxf(tmax, X(c));
             }
-            if (j == nkv - 1) {
-                const int valid = N - j * kBN;
-                if (valid < kBN) {
-#pragma unroll
-                    for (int c = 0; c < kBN; ++c)
-                        if (c >= valid) x[c] = -INFINITY;
-                }
-            }
-            // Row max over the tile: 8 independent chains of 3-input max.
-            float mx[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = x[i];
-#pragma unroll
-            for (int c = 8; c < kBN; c += 16)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], x[c + i], x[c + 8 + i]);
-            const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
             const float m_new = fmaxf(m, tmax * scale_log2);
             if (j == 0) {
                 m = m_new;
@@ -344,20 +361,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
                     const float2 alpha2 = make_float2(alpha, alpha);
-                    uint32_t r[32];
+                    uint32_t ro[32];
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
-                        tmem_ld32(tO + c * 32, r);
+                        tmem_ld32(tO + c * 32, ro);
                         tmem_wait_ld();
-                        reg_fence32(r);
+                        reg_fence32(ro);
 #pragma unroll
                         for (int i = 0; i < 32; i += 2) {
                             const float2 v = __fmul2_rn(
-                                make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), alpha2);
-                            r[i] = __float_as_uint(v.x);
-                            r[i + 1] = __float_as_uint(v.y);
+                                make_float2(__uint_as_float(ro[i]), __uint_as_float(ro[i + 1])), alpha2);
+                            ro[i] = __float_as_uint(v.x);
+                            ro[i + 1] = __float_as_uint(v.y);
                         }
-                        tmem_st32(tO + c * 32, r);
+                        tmem_st32(tO + c * 32, ro);
                     }
                     tmem_wait_st();
                     if (need) {
@@ -366,29 +383,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            // P = 2^(s·scale·log2e − m): packed FFMA, MUFU ex2, packed row sum.
+            // P = 2^(s·scale·log2e − m): packed FFMA, ex2 (MUFU, or the FMA
+            // pipe for kEmuOf8 pairs in 8), packed row sum, bf16 pairs into
+            // tensor memory.  Each 64-key half is published as soon as it is
+            // written, so its P·V MMAs start while the next half is computed.
+            // Keys past N get P = 0.
             const float2 c2 = make_float2(scale_log2, scale_log2);
             const float2 negm2 = make_float2(-m, -m);
             float2 ls[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            auto exp_half = [&](int hf, auto tail_tag) {
+                constexpr bool kTail = decltype(tail_tag)::value;
                 uint32_t p[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float2 t = __ffma2_rn(make_float2(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]), c2, negm2);
-                    const float2 e = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                    const int col = hf * 64 + 2 * i;
+                    const float2 t = __ffma2_rn(make_float2(X(col), X(col + 1)), c2, negm2);
+                    float2 e;
+                    if (!kTail && (i & 7) < kEmuOf8)
+                        e = exp2_poly2(t);
+                    else
+                        e = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                    if (kTail) {
+                        if (col >= valid) e.x = 0.f;
+                        if (col + 1 >= valid) e.y = 0.f;
+                    }
                     ls[i & 3] = __fadd2_rn(ls[i & 3], e);
                     p[i] = pack_bf16x2(e.x, e.y);
                 }
-                tmem_st32(tS + c * 32, p);
+                tmem_st32(tS + hf * 32, p);
+                if (kSplitP || hf == 1) {
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&bars.p_full[2 * wg + (kSplitP ? hf : 0)]);
+                }
+            };
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                if (valid < kBN)
+                    exp_half(hf, std::true_type{});
+                else
+                    exp_half(hf, std::false_type{});
             }
             const float2 lsum = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
             l += lsum.x + lsum.y;
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bars.p_full[wg]);
         }
         // Epilogue: O / l -> bf16 -> global (rows at or past N are padding).
         if (ok) ok = mbar_wait(&bars.o_ready[wg], (nkv - 1) & 1, abort_flag, err);

@@ -62,6 +62,7 @@ struct Q8Cfg {
     static constexpr uint32_t kIdescPV = FP8 ? make_idesc(1, 0, 0, 0, 1, 128, D) : make_idesc(1, 1, 1, 0, 1, 128, D);
     static constexpr float kShift = FP8 ? 6.5f : 0.0f;     // log2 of P's scale
     static constexpr float kThresh = FP8 ? 2.0f : 8.0f;    // rescale threshold (log2)
+    static constexpr int kEmuOf8 = 0;                      // exp2 pairs (of 8) on the FMA pipe
 };
 
 struct Bars {
@@ -83,25 +84,6 @@ __device__ __forceinline__ Bars carve(uint8_t* base) {
     r.o_ready = r.p_full + 2;
     r.mma_done = r.o_ready + 2;
     return r;
-}
-
-__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
-        : "memory");
-}
-__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc)
-        : "memory");
 }
 
 // Four fp32 -> four e4m3 in one word (round to nearest even, saturating);
@@ -212,57 +194,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else if (warp == kMmaWarp) {
             // -------------------------------------------------------- MMA issuer
-            const uint32_t sQ0 = smem_base + C::kQOff;
-            const uint32_t sQ1 = sQ0 + C::kQTile;
-            const uint32_t tS0 = tmem, tS1 = tmem + 128;
-            const uint32_t tO0 = tmem + 256, tO1 = tmem + 384;
-            // K-major int8 operand, k-step kk = 32 bytes inside the 128-B swizzled row.
-            auto desc_k = [](uint32_t tile, int kk) { return smem_desc_sw128(tile + kk * 32, 16, 1024); };
+            // Descriptors are built once and advanced by byte offsets (SDesc).
+            // K-major int8 operand: k-step kk = 32 bytes inside the 128-B row.
             // V, MN-major: FP8 rows are one 128-B panel (k-step 32 keys);
             // bf16 is two 64-element panels 16 KB apart (k-step 16 keys).
-            auto desc_v = [](uint32_t tile, int kk) {
-                return FP8 ? smem_desc_sw128(tile + kk * 32 * 128, kPanel, 1024)
-                           : smem_desc_sw128(tile + kk * 16 * 128, kPanel, 1024);
-            };
+            const SDesc dQ0 = sdesc_sw128(smem_base + C::kQOff, 16, 1024);
+            const SDesc dQ1 = sdesc_add(dQ0, C::kQTile);
+            const SDesc dK0 = sdesc_sw128(smem_base + C::kKOff, 16, 1024);
+            const SDesc dV0 = sdesc_sw128(smem_base + C::kVOff, kPanel, 1024);
+            const uint32_t tS0 = tmem, tS1 = tmem + 128;
+            const uint32_t tO0 = tmem + 256, tO1 = tmem + 384;
             constexpr int kQKSteps = D / 32;
             constexpr int kPVSteps = FP8 ? kBN / 32 : kBN / 16;
-            auto issue_s = [&](uint32_t tS, uint32_t sQ, uint32_t sK) {
+            constexpr uint32_t kVStep = FP8 ? 32 * 128 : 16 * 128;
+            auto issue_s = [&](uint32_t tS, SDesc dQ, SDesc dK) {
 #pragma unroll
-                for (int kk = 0; kk < kQKSteps; ++kk) mma_i8_ss(tS, desc_k(sQ, kk), desc_k(sK, kk), C::kIdescQK, kk > 0);
+                for (int kk = 0; kk < kQKSteps; ++kk)
+                    mma_ss<1>(tS, sdesc_add(dQ, kk * 32), sdesc_add(dK, kk * 32), C::kIdescQK, kk > 0);
             };
-            auto issue_pv = [&](uint32_t tO, uint32_t tP, uint32_t sV, bool acc) {
+            auto issue_pv = [&](uint32_t tO, uint32_t tP, SDesc dV, bool acc) {
 #pragma unroll
-                for (int kk = 0; kk < kPVSteps; ++kk) {
-                    if (FP8)
-                        mma_f8_ts(tO, tP + kk * 8, desc_v(sV, kk), C::kIdescPV, acc || kk > 0);
-                    else
-                        mma_bf16_ts(tO, tP + kk * 8, desc_v(sV, kk), C::kIdescPV, acc || kk > 0);
-                }
+                for (int kk = 0; kk < kPVSteps; ++kk)
+                    mma_ts<FP8 ? 2 : 0>(tO, tP + kk * 8, sdesc_add(dV, kk * kVStep), C::kIdescPV, acc || kk > 0);
             };
             bool ok = mbar_wait(bars.q_full, 0, abort_flag, err) && mbar_wait(&bars.k_full[0], 0, abort_flag, err);
             if (ok) {
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t sK = smem_base + C::kKOff;
-                    issue_s(tS0, sQ0, sK);
+                    issue_s(tS0, dQ0, dK0);
                     mma_commit(&bars.s_full[0]);
-                    issue_s(tS1, sQ1, sK);
+                    issue_s(tS1, dQ1, dK0);
                     mma_commit(&bars.s_full[1]);
                     mma_commit(&bars.k_empty[0]);
                 }
                 __syncwarp();
                 for (int j = 0; j < nkv && ok; ++j) {
                     const int vs = j % C::kStages;
-                    const uint32_t sV = smem_base + C::kVOff + vs * C::kVTile;
+                    const SDesc dV = sdesc_add(dV0, vs * C::kVTile);
                     const bool more = j + 1 < nkv;
                     const int ks = (j + 1) % C::kStages;
-                    const uint32_t sK = smem_base + C::kKOff + ks * C::kKTile;
+                    const SDesc dK = sdesc_add(dK0, ks * C::kKTile);
                     ok = mbar_wait(&bars.v_full[vs], (j / C::kStages) & 1, abort_flag, err) &&
                          mbar_wait(&bars.p_full[0], j & 1, abort_flag, err);
                     if (!ok) break;
                     tc_fence_after();
                     if (lane == 0) {
-                        issue_pv(tO0, tS0, sV, j > 0);
+                        issue_pv(tO0, tS0, dV, j > 0);
                         mma_commit(&bars.o_ready[0]);
                     }
                     __syncwarp();
@@ -271,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) break;
                         tc_fence_after();
                         if (lane == 0) {
-                            issue_s(tS0, sQ0, sK);
+                            issue_s(tS0, dQ0, dK);
                             mma_commit(&bars.s_full[0]);
                         }
                         __syncwarp();
@@ -280,11 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc_fence_after();
                     if (lane == 0) {
-                        issue_pv(tO1, tS1, sV, j > 0);
+                        issue_pv(tO1, tS1, dV, j > 0);
                         mma_commit(&bars.o_ready[1]);
                         mma_commit(&bars.v_empty[vs]);
                         if (more) {
-                            issue_s(tS1, sQ1, sK);
+                            issue_s(tS1, dQ1, dK);
                             mma_commit(&bars.s_full[1]);
                             mma_commit(&bars.k_empty[ks]);
                         }
@@ -405,8 +382,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float2 f = make_float2(__int_as_float(static_cast<int>(r[i >> 5][i & 31]) + 0x4B400000),
                                              __int_as_float(static_cast<int>(r[(i + 1) >> 5][(i + 1) & 31]) + 0x4B400000));
                 const float2 t = __ffma2_rn(f, cc, nb);
-                p[i] = ex2_approx(t.x);
-                p[i + 1] = ex2_approx(t.y);
+                if (((i >> 1) & 7) < C::kEmuOf8) {
+                    const float2 e = exp2_poly2(t);
+                    p[i] = e.x;
+                    p[i + 1] = e.y;
+                } else {
+                    p[i] = ex2_approx(t.x);
+                    p[i + 1] = ex2_approx(t.y);
+                }
             }
             if (tail) {
 #pragma unroll

@@ -183,6 +183,63 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t dfmt, uint32_t afmt, 
            ((M >> 4) << 24);
 }
 
+// Shared-memory descriptors are passed as (low word, high word).  The start
+// address lives in bits 0-13 of the low word in 16-byte units, so a
+// descriptor for the same layout `bytes` further on is lo + bytes/16 (shared
+// memory ends below 2^18 bytes: no carry leaves the field).  Building every
+// descriptor once and advancing only its low word keeps the issuing thread's
+// per-MMA work to one add, so MMAs issue at the tensor core's rate.
+struct SDesc {
+    uint32_t lo, hi;
+};
+__device__ __forceinline__ SDesc sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    const uint64_t d = smem_desc_sw128(saddr, lbo_bytes, sbo_bytes);
+    return SDesc{static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
+}
+__device__ __forceinline__ SDesc sdesc_add(SDesc d, uint32_t bytes) { return SDesc{d.lo + (bytes >> 4), d.hi}; }
+
+// D[tmem] (+)= A[smem] · B[smem] (kind::f16 / kind::i8), split descriptors.
+template <int KIND>  // 0: f16 (bf16 in, fp32 acc), 1: i8 (s8 in, s32 acc)
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, SDesc a, SDesc b, uint32_t idesc, uint32_t accumulate) {
+    if (KIND == 0)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+            "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+            "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+            "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+            "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
+            : "memory");
+}
+// D[tmem] (+)= A[tmem] · B[smem] (kind::f16 / kind::f8f6f4), split descriptor.
+template <int KIND>  // 0: f16, 2: f8f6f4
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, SDesc b, uint32_t idesc,
+                                       uint32_t accumulate) {
+    if (KIND == 0)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+            "mov.b64 db, {%2, %3};\n\t"
+            "setp.ne.b32 p, %5, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+            "r"(a_tmem), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+            "mov.b64 db, {%2, %3};\n\t"
+            "setp.ne.b32 p, %5, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+            "r"(a_tmem), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
+            : "memory");
+}
+
 // D[tmem] (+)= A[smem] · B[smem], bf16 inputs, fp32 accumulate.
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -235,6 +292,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// 2^x for a pair of floats on the FMA pipe instead of MUFU.  Cody–Waite
+// split x = j + r with j = round(x) (adding 1.5·2^23 leaves j in the low
+// mantissa bits) and |r| <= 1/2; 2^r from a cubic (relative-error minimax on
+// [-1/2, 1/2], fitted for this library, max relative error 7.5e-5, far below
+// bf16's 2^-9); then j is added to the exponent field.  x is clamped at -125
+// so the result stays a normal float (2^-125 stands in for anything smaller).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+    const float2 jf = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 r = __ffma2_rn(jf, make_float2(-1.f, -1.f), x);
+    float2 p = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), r, make_float2(0.2426111251f, 0.2426111251f));
+    p = __ffma2_rn(p, r, make_float2(0.6932609677f, 0.6932609677f));
+    p = __ffma2_rn(p, r, make_float2(0.9999280572f, 0.9999280572f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` goes to bits 0-15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
