@@ -62,7 +62,7 @@ struct Q8Cfg {
     static constexpr uint32_t kIdescPV = FP8 ? make_idesc(1, 0, 0, 0, 1, 128, D) : make_idesc(1, 1, 1, 0, 1, 128, D);
     static constexpr float kShift = FP8 ? 6.5f : 0.0f;     // log2 of P's scale
     static constexpr float kThresh = FP8 ? 2.0f : 8.0f;    // rescale threshold (log2)
-    static constexpr int kEmuOf8 = 0;                      // exp2 pairs (of 8) on the FMA pipe
+    static constexpr int kEmuOf8 = FP8 ? 2 : 1;            // exp2 pairs (of 8) on the FMA pipe (tuned)
 };
 
 struct Bars {
