@@ -45,6 +45,11 @@ METRIC = "attention TFLOPS (4·B·H·N²·d/s) and % of B200 tensor peak at N=11
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
+# DRAM bytes (read + write) of one launch, from the ncu capture summarised in
+# profiles/attn_fwd_bf16_video_mid_n45760.md (N=45760, 24 heads), scaled by N:
+# each head's K/V stays L2-resident while its CTAs run, so traffic grows with N.
+# Set to None whenever the kernel changes until it is captured again.
+BF16_ATTN_DRAM_BYTES_AT = (1.134775e9, 45760)
 SPEC_HBM_GBS = 8000.0
 
 
@@ -130,6 +135,22 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def max_over_ranks(values, device, world_size: int):
+    """Element-wise max of a list of floats over all ranks (timings: the job
+    takes as long as its slowest rank).  One all-reduce; no-op on one rank."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world_size > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def rank_case(base: inputs.AttnCase, rank: int) -> inputs.AttnCase:
+    """The workload replica of one rank: same shape, inputs seeded by rank."""
+    return inputs.AttnCase(base.name, base.B, base.H, base.N, base.d, k_offset_std=base.k_offset_std, seed=rank)
 
 
 def pinned_bf16(bits: np.ndarray):
@@ -233,7 +254,7 @@ def run_ours(args):
             dist.barrier()
 
     base = WORKLOADS[args.workload]
-    case = inputs.AttnCase(base.name, base.B, base.H, base.N, base.d, k_offset_std=base.k_offset_std, seed=rank)
+    case = rank_case(base, rank)
     fcase = inputs.FbcCase(f"fbc_{base.N}x{base.H * base.d}_bf16", base.N, base.H * base.d, "bf16", 0.03, 0.08,
                            seed=rank)
     q, k, v = inputs.attn_inputs(case)
@@ -350,10 +371,8 @@ def run_ours(args):
     prepass_ms = ep[0].elapsed_time(ep[1]) / K
 
     # ---- max over ranks
-    t = torch.tensor([ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms = t.tolist()
+    ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms = max_over_ranks(
+        [ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms], dev, ws)
 
     flops = 4.0 * case.B * case.H * case.N * case.N * case.d  # one attention call
     value = ws * K * 2 * flops / (ms * 1e-3) / 1e12
@@ -387,7 +406,12 @@ def run_ours(args):
         "clocks": clocks,
     }
     roof_bf16 = {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
-                 "frac": attn_tflops / peak, "traffic": None, "kernel": "attn_fwd_bf16_kernel<128>",
+                 "frac": attn_tflops / peak,
+                 "traffic": (BF16_ATTN_DRAM_BYTES_AT[0] * case.N / BF16_ATTN_DRAM_BYTES_AT[1] * case.B * case.H / 24
+                             if BF16_ATTN_DRAM_BYTES_AT else None),
+                 "traffic_unit": "bytes per launch (ncu, scaled by N from the 45760-token capture)",
+                 "algorithmic_bytes": 4.0 * case.B * case.H * case.N * case.d * 2,
+                 "kernel": "attn_fwd_bf16_kernel<128>",
                  "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
                  "frac_of_spec_2250": attn_tflops / SPEC_BF16_TFLOPS}
     roof_q8 = {"bound": "tensor", "achieved": q8_attn_tflops, "peak": peak8, "unit": "TFLOP/s",
