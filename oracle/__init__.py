@@ -192,3 +192,47 @@ def emulated_q8_attention(q, k, v, scale: float | None = None, smooth_k: bool = 
     kd = kc.astype(np.float64) * ks[:, :, tok // 64, None].astype(np.float64)
     vd = e4m3_decode(vc).astype(np.float64) * vs[:, :, None, :].astype(np.float64)
     return attention(qd, kd, vd, scale=scale, rows=rows)
+
+
+def _widen(x) -> np.ndarray:
+    """fp32 array, or uint16 array of bf16 bits, to fp64 (exact)."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if x.dtype in (np.float32, np.float64):
+        return x.astype(np.float64)
+    raise TypeError(x.dtype)
+
+
+def compare_stats(ref, test, segments: int = 1):
+    """Error of ``test`` against ``ref`` per contiguous segment, in fp64.
+
+    TMAP image-to-video page, "keeping video quality": the attention error of
+    each layer over the denoising steps is what singles out the layers whose
+    8-bit attention is switched back to 16 bits.  The error measures are the
+    relative L1 distance sum|test - ref| / sum|ref|, the cosine similarity
+    sum(ref*test) / sqrt(sum(ref^2) sum(test^2)) and max|test - ref|.
+    Both inputs are fp32 arrays or uint16 arrays of bf16 bits with the same
+    number of elements, which ``segments`` divides.  Conventions for empty
+    norms: rel_l1 is 0 if both sums are 0 and +inf if only sum|ref| is;
+    cosine is 1 if both vectors are zero and 0 if exactly one is.
+    Returns three float64 arrays of length ``segments``.
+    """
+    a = _widen(ref).reshape(segments, -1)
+    b = _widen(test).reshape(segments, -1)
+    assert a.shape == b.shape
+    rel = np.empty(segments)
+    cos = np.empty(segments)
+    mx = np.empty(segments)
+    for s in range(segments):
+        x, y = a[s], b[s]
+        num = np.abs(y - x).sum()
+        den = np.abs(x).sum()
+        rel[s] = num / den if den > 0 else (np.inf if num > 0 else 0.0)
+        xx, yy, xy = (x * x).sum(), (y * y).sum(), (x * y).sum()
+        if xx > 0 and yy > 0:
+            cos[s] = xy / np.sqrt(xx * yy)
+        else:
+            cos[s] = 1.0 if (xx == 0 and yy == 0) else 0.0
+        mx[s] = np.abs(y - x).max() if x.size else 0.0
+    return rel, cos, mx
