@@ -12,7 +12,12 @@ Entry points (same names as the C ABI in ``include/dit_attn.h``):
   * ``dit_attn_q8_quantize(q, k, v, ...)``         — its pre-pass alone
   * ``fbc_rel_l1(r_cur, r_prev, threshold, ...)``   — first-block-cache decision
   * ``fbc_rel_l1_noalloc(...)``                     — the same, allocating nothing
+  * ``dit_compare_stats(ref, test, segments)``       — rel-L1 / cosine / max error per segment
   * ``dit_get_device_status()``                     — device-side error word
+
+and of ``include/dit_cache.h``:
+  * ``fbcache_step(...)`` / ``teacache_step(...)``  — step-cache decisions kept on the device
+  * ``dit_cache_state_reset``, ``dit_graph_*``     — device state and CUDA-graph conditional plumbing
 """
 from __future__ import annotations
 
@@ -49,8 +54,23 @@ SIGNATURES = {
     "fbc_rel_l1_workspace_bytes": (_sz, [_i64]),
     "fbc_rel_l1": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p, _sz, _p]),
     "fbc_rel_l1_noalloc": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p]),
+    "dit_compare_workspace_bytes": (_sz, [_i64, _i64, _i]),
+    "dit_compare_stats": (_i, [_p, _p, _i64, _i64, _i, _p, _p, _sz, _p]),
     "dit_get_device_status": (_i, [_p]),
     "dit_status_string": (ctypes.c_char_p, [_i]),
+    # include/dit_cache.h
+    "dit_cache_state_reset": (_i, [_p, _p]),
+    "dit_cache_workspace_bytes": (_sz, [_i64]),
+    "fbcache_step": (_i, [_p, _p, _i64, _i, _p, _p, _p, ctypes.c_int32, _i, ctypes.c_ulonglong, _p, _sz, _p]),
+    "teacache_step": (_i, [_p, _p, _i64, _i, _p, ctypes.c_int32, _f, _p, _p, ctypes.c_int32, _i,
+                           ctypes.c_ulonglong, _p, _sz, _p]),
+    "dit_graph_capture_begin": (_i, [_p]),
+    "dit_graph_cond_create": (_i, [_p, _p]),
+    "dit_graph_cond_body_begin": (_i, [_p, ctypes.c_ulonglong, _p]),
+    "dit_graph_cond_body_end": (_i, [_p]),
+    "dit_graph_capture_end": (_i, [_p, _p]),
+    "dit_graph_launch": (_i, [_p, _p]),
+    "dit_graph_destroy": (_i, [_p]),
 }
 
 _lib = None
@@ -278,3 +298,183 @@ def fbc_rel_l1_noalloc(r_cur, r_prev, threshold: float, out_rel, out_skip, strea
 def dit_get_device_status(stream=None) -> int:
     """Synchronise the stream; return (and clear) the device error word."""
     return int(load_library().dit_get_device_status(_stream_ptr(stream)))
+
+
+def dit_compare_workspace_bytes(n_segments: int, segment_len: int, dtype) -> int:
+    return int(load_library().dit_compare_workspace_bytes(int(n_segments), int(segment_len), int(dtype)))
+
+
+def _dtype_code(t, what):
+    import torch
+    dt = {torch.float32: DIT_DTYPE_F32, torch.bfloat16: DIT_DTYPE_BF16}.get(t.dtype)
+    if dt is None:
+        raise TypeError(f"{what} expects fp32 or bf16 tensors")
+    return dt
+
+
+def dit_compare_stats(ref, test, segments: int = 1, out=None, workspace=None, stream=None):
+    """Error of ``test`` against ``ref`` per contiguous segment, on the device.
+
+    Returns a float64 device tensor [segments, 3]: relative L1, cosine
+    similarity, max abs difference.  No host synchronisation.
+    """
+    import torch
+    lib = load_library()
+    if ref.shape != test.shape or ref.dtype != test.dtype:
+        raise ValueError("ref and test must match in shape and dtype")
+    if not (ref.is_contiguous() and test.is_contiguous()):
+        raise ValueError("ref and test must be contiguous")
+    dt = _dtype_code(ref, "dit_compare_stats")
+    n = ref.numel()
+    if segments < 1 or n % segments:
+        raise ValueError("segments must divide the element count")
+    seg_len = n // segments
+    if out is None:
+        out = torch.empty(segments, 3, dtype=torch.float64, device=ref.device)
+    if workspace is None:
+        workspace = torch.zeros(dit_compare_workspace_bytes(segments, seg_len, dt), dtype=torch.uint8,
+                                device=ref.device)
+    st = lib.dit_compare_stats(ref.data_ptr(), test.data_ptr(), segments, seg_len, dt, out.data_ptr(),
+                               workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(st, "dit_compare_stats")
+    return out
+
+
+# ---- step caches (include/dit_cache.h) ------------------------------------
+
+DIT_CACHE_USE = 0
+DIT_CACHE_WARMUP = 1
+DIT_CACHE_NO_PREV = 2
+DIT_CACHE_ABOVE_THRESHOLD = 3
+DIT_CACHE_MAX_CACHED = 4
+DIT_CACHE_MAX_CONTINUOUS = 5
+CACHE_STATE_BYTES = 40
+CACHE_TRACE_BYTES = 24
+
+
+class dit_cache_policy(ctypes.Structure):
+    """Policy of fbcache_step; defaults of the DiffusionCacheConfig table."""
+    _fields_ = [("max_warmup_steps", ctypes.c_int32), ("max_cached_steps", ctypes.c_int32),
+                ("max_continuous_cached_steps", ctypes.c_int32), ("residual_diff_threshold", ctypes.c_float)]
+
+    def __init__(self, max_warmup_steps=4, max_cached_steps=-1, max_continuous_cached_steps=3,
+                 residual_diff_threshold=0.24):
+        super().__init__(int(max_warmup_steps), int(max_cached_steps), int(max_continuous_cached_steps),
+                         float(residual_diff_threshold))
+
+
+def cache_state(device=None):
+    """A fresh (zeroed) device-resident dit_cache_state."""
+    import torch
+    return torch.zeros(CACHE_STATE_BYTES, dtype=torch.uint8, device=device or "cuda")
+
+
+def cache_trace(capacity: int, device=None):
+    import torch
+    return torch.zeros(int(capacity) * CACHE_TRACE_BYTES, dtype=torch.uint8, device=device or "cuda")
+
+
+def read_cache_state(state) -> dict:
+    """Copy a dit_cache_state to the host (synchronises)."""
+    import numpy as np
+    b = state.detach().cpu().numpy().tobytes()
+    i = np.frombuffer(b[:24], dtype=np.int32)
+    f = np.frombuffer(b[24:40], dtype=np.float64)
+    return {"step": int(i[0]), "cached_steps": int(i[1]), "continuous_cached": int(i[2]),
+            "has_prev": int(i[3]), "last_decision": int(i[4]), "last_rel": float(f[0]), "acc": float(f[1])}
+
+
+def read_cache_trace(trace, count: int):
+    """First ``count`` trace entries as a numpy record array (rel, acc, decision)."""
+    import numpy as np
+    dt = np.dtype([("rel", "<f8"), ("acc", "<f8"), ("decision", "<i4"), ("reserved", "<i4")])
+    return np.frombuffer(trace.detach().cpu().numpy().tobytes(), dtype=dt)[:count]
+
+
+def dit_cache_workspace_bytes(n: int) -> int:
+    return int(load_library().dit_cache_workspace_bytes(int(n)))
+
+
+def cache_workspace(n: int, device=None):
+    import torch
+    return torch.zeros(dit_cache_workspace_bytes(n), dtype=torch.uint8, device=device or "cuda")
+
+
+def dit_cache_state_reset(state, stream=None):
+    _check(load_library().dit_cache_state_reset(state.data_ptr(), _stream_ptr(stream)), "dit_cache_state_reset")
+
+
+def _step_args(cur, prev, what):
+    if cur.shape != prev.shape or cur.dtype != prev.dtype:
+        raise ValueError(f"{what}: inputs must match in shape and dtype")
+    if not (cur.is_contiguous() and prev.is_contiguous()):
+        raise ValueError(f"{what}: inputs must be contiguous")
+    return _dtype_code(cur, what)
+
+
+def fbcache_step(r_cur, r_prev, policy: dit_cache_policy, state, trace=None, cond_handle=None, workspace=None,
+                 stream=None):
+    """One first-block-cache decision; updates ``state`` on the device."""
+    lib = load_library()
+    dt = _step_args(r_cur, r_prev, "fbcache_step")
+    n = r_cur.numel()
+    if workspace is None:
+        workspace = cache_workspace(n, r_cur.device)
+    cap = trace.numel() // CACHE_TRACE_BYTES if trace is not None else 0
+    st = lib.fbcache_step(r_cur.data_ptr(), r_prev.data_ptr(), n, dt, ctypes.byref(policy), state.data_ptr(),
+                          trace.data_ptr() if trace is not None else None, cap,
+                          0 if cond_handle is None else 1, 0 if cond_handle is None else int(cond_handle),
+                          workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(st, "fbcache_step")
+    return state
+
+
+def teacache_step(x_cur, x_prev, coeffs, threshold: float, state, trace=None, cond_handle=None, workspace=None,
+                  stream=None):
+    """One TeaCache decision; updates ``state`` and stores x_cur into x_prev."""
+    lib = load_library()
+    dt = _step_args(x_cur, x_prev, "teacache_step")
+    n = x_cur.numel()
+    if workspace is None:
+        workspace = cache_workspace(n, x_cur.device)
+    c = (ctypes.c_double * len(coeffs))(*[float(v) for v in coeffs])
+    cap = trace.numel() // CACHE_TRACE_BYTES if trace is not None else 0
+    st = lib.teacache_step(x_cur.data_ptr(), x_prev.data_ptr(), n, dt, c, len(coeffs), float(threshold),
+                           state.data_ptr(), trace.data_ptr() if trace is not None else None, cap,
+                           0 if cond_handle is None else 1, 0 if cond_handle is None else int(cond_handle),
+                           workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(st, "teacache_step")
+    return state
+
+
+def dit_graph_capture_begin(stream):
+    _check(load_library().dit_graph_capture_begin(_stream_ptr(stream)), "dit_graph_capture_begin")
+
+
+def dit_graph_cond_create(stream) -> int:
+    h = ctypes.c_ulonglong(0)
+    _check(load_library().dit_graph_cond_create(_stream_ptr(stream), ctypes.byref(h)), "dit_graph_cond_create")
+    return int(h.value)
+
+
+def dit_graph_cond_body_begin(stream, cond_handle: int, body_stream):
+    _check(load_library().dit_graph_cond_body_begin(_stream_ptr(stream), int(cond_handle), _stream_ptr(body_stream)),
+           "dit_graph_cond_body_begin")
+
+
+def dit_graph_cond_body_end(body_stream):
+    _check(load_library().dit_graph_cond_body_end(_stream_ptr(body_stream)), "dit_graph_cond_body_end")
+
+
+def dit_graph_capture_end(stream) -> int:
+    g = ctypes.c_void_p(0)
+    _check(load_library().dit_graph_capture_end(_stream_ptr(stream), ctypes.byref(g)), "dit_graph_capture_end")
+    return int(g.value)
+
+
+def dit_graph_launch(graph_exec: int, stream):
+    _check(load_library().dit_graph_launch(ctypes.c_void_p(graph_exec), _stream_ptr(stream)), "dit_graph_launch")
+
+
+def dit_graph_destroy(graph_exec: int):
+    _check(load_library().dit_graph_destroy(ctypes.c_void_p(graph_exec)), "dit_graph_destroy")

@@ -17,8 +17,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libditattn.so")
 
-SOURCES = ["api.cu", "attn_bf16.cu", "attn_q8.cu", "q8_prepass.cu", "fbc_rel_l1.cu"]
-HEADERS = ["sm100_ptx.cuh", "internal.h"]
+SOURCES = ["api.cu", "attn_bf16.cu", "attn_q8.cu", "q8_prepass.cu", "fbc_rel_l1.cu", "cache_step.cu",
+           "compare.cu"]
+HEADERS = ["sm100_ptx.cuh", "internal.h", "rel_l1_reduce.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -38,7 +39,7 @@ def nvcc_path() -> str:
 
 def _inputs():
     files = [os.path.join(CSRC, s) for s in SOURCES + HEADERS]
-    files.append(os.path.join(INCLUDE, "dit_attn.h"))
+    files += [os.path.join(INCLUDE, h) for h in sorted(os.listdir(INCLUDE)) if h.endswith(".h")]
     return files
 
 

@@ -1,7 +1,8 @@
 // C ABI of libditattn.so (declared in include/dit_attn.h): argument
 // validation, TMA tensor-map encoding and launches.  Host code only; the
 // arithmetic of every call runs in the kernels of attn_bf16.cu, attn_q8.cu,
-// q8_prepass.cu and fbc_rel_l1.cu.
+// q8_prepass.cu and fbc_rel_l1.cu (the step caches and the output comparison
+// have their own entry points in cache_step.cu and compare.cu).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -160,6 +161,13 @@ dit_status check_q8_args(int d, int smooth_k, int pv_mode, const void* ws, size_
 }
 
 }  // namespace
+
+dit_status check_device() {
+    dit_status st;
+    device_state(&st);
+    return st;
+}
+
 }  // namespace ditk
 
 using namespace ditk;

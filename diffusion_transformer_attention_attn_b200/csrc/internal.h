@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "dit_attn.h"
+
 namespace ditk {
 
 // Softmax attention, bf16 in/out.  tq/tk/tv: 4-D tensor maps {d, N, H, B} with
@@ -38,6 +40,10 @@ cudaError_t launch_q8_prepass(const void* q, const void* k, const void* v, int64
 cudaError_t launch_attn_q8(const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv, int pv_fp8,
                            const uint8_t* ws, const Q8Layout& L, void* o, int64_t sb, int64_t sh, int64_t sn, int B,
                            int H, int N, float scale_log2, int* err, cudaStream_t stream);
+
+// DIT_OK when the current device is an sm_100 part (its one-time set-up done),
+// else DIT_ERR_UNSUPPORTED or DIT_ERR_CUDA.
+dit_status check_device();
 
 // First-block-cache residual difference (see fbc_rel_l1 in dit_attn.h).
 size_t fbc_workspace_bytes(int64_t n);

@@ -1,0 +1,205 @@
+// One-pass relative-L1 reduction shared by the step-caching calls.
+//
+// Each call computes num = Σ|cur − prev| and den = Σ|prev| over n elements in
+// a single launch and hands the two sums to an epilogue run by thread 0 of the
+// last block to finish:
+//   * EpiThreshold (fbc_rel_l1): rel = num/den and skip = rel < threshold.
+//   * the step policies of cache_step.cu, which also keep device-resident
+//     counters and may set a CUDA-graph conditional.
+//
+// HBM-bound streaming: every thread reads 16-byte vectors of both inputs
+// (grid-stride, four vectors of each in flight), sums in fp32 over at most 32
+// elements and folds into fp64; blocks reduce in fp64 with warp shuffles.
+// Each block writes its partial pair to the workspace; the last block to take
+// a ticket adds the partials in block order, runs the epilogue and re-zeroes
+// the ticket.  The grid size depends on n only, so the summation order, and
+// the result, are the same on every run.
+//
+// With kCopy the kernel also stores cur into prev in the same pass (each
+// element is read before the same thread overwrites it), the update that the
+// TeaCache accumulator needs on every step.  An epilogue may declare that the
+// sums are not needed (evaluate() false): the kernel then reads nothing and
+// only runs the epilogue.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+namespace ditk {
+
+constexpr int kFbcThreads = 512;
+constexpr int kFbcMaxBlocks = 1024;
+constexpr int kFbcUnroll = 4;
+
+struct FbcWs {
+    unsigned int ticket;
+    unsigned int pad[3];
+    // followed by double2 partials[kFbcMaxBlocks]
+};
+
+__device__ __forceinline__ void rl1_acc(const float4& c, const float4& p, float& num, float& den) {
+    num += fabsf(c.x - p.x) + fabsf(c.y - p.y) + fabsf(c.z - p.z) + fabsf(c.w - p.w);
+    den += fabsf(p.x) + fabsf(p.y) + fabsf(p.z) + fabsf(p.w);
+}
+__device__ __forceinline__ float rl1_bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float rl1_bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+__device__ __forceinline__ void rl1_acc(const uint4& c, const uint4& p, float& num, float& den) {
+    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float c0 = rl1_bf_lo(cw[i]), c1 = rl1_bf_hi(cw[i]);
+        const float p0 = rl1_bf_lo(pw[i]), p1 = rl1_bf_hi(pw[i]);
+        num += fabsf(c0 - p0) + fabsf(c1 - p1);
+        den += fabsf(p0) + fabsf(p1);
+    }
+}
+
+__device__ __forceinline__ double rl1_warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Deterministic block sum of (a, b) in fp64; result valid in thread 0.
+__device__ __forceinline__ void rl1_block_sum2(double& a, double& b, double2* sh) {
+    a = rl1_warp_sum(a);
+    b = rl1_warp_sum(b);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) sh[warp] = make_double2(a, b);
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        double2 v = lane < nw ? sh[lane] : make_double2(0.0, 0.0);
+        a = rl1_warp_sum(v.x);
+        b = rl1_warp_sum(v.y);
+    }
+}
+
+// rel = num / den; den = 0 gives 0 when num = 0 too, else +inf.
+__device__ __forceinline__ double rl1_ratio(double num, double den) {
+    if (den > 0.0) return num / den;
+    return num > 0.0 ? HUGE_VAL : 0.0;
+}
+
+// VecT: float4 (fp32 inputs, 4 elements) or uint4 (bf16 inputs, 8 elements).
+template <typename VecT, int kElems, bool kCopy, typename Epi>
+__global__ void __launch_bounds__(kFbcThreads)
+    rel_l1_kernel(const VecT* __restrict__ cur, VecT* prev, int64_t nvec, const void* __restrict__ cur_tail,
+                  void* prev_tail, int tail, Epi epi, FbcWs* ws) {
+    __shared__ double2 sh[kFbcThreads / 32];
+    __shared__ bool is_last;
+    double2* partials = reinterpret_cast<double2*>(ws + 1);
+    const bool eval = epi.evaluate();
+
+    double num = 0.0, den = 0.0;
+    if (eval || kCopy) {
+        const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+        int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+        for (; i + (kFbcUnroll - 1) * stride < nvec; i += kFbcUnroll * stride) {
+            VecT c[kFbcUnroll], p[kFbcUnroll];
+#pragma unroll
+            for (int u = 0; u < kFbcUnroll; ++u) {
+                c[u] = __ldcs(cur + i + u * stride);
+                p[u] = __ldcs(prev + i + u * stride);
+            }
+            if (kCopy) {
+#pragma unroll
+                for (int u = 0; u < kFbcUnroll; ++u) __stcs(prev + i + u * stride, c[u]);
+            }
+            float fn = 0.f, fd = 0.f;
+#pragma unroll
+            for (int u = 0; u < kFbcUnroll; ++u) rl1_acc(c[u], p[u], fn, fd);
+            num += fn;
+            den += fd;
+        }
+        for (; i < nvec; i += stride) {
+            const VecT c = __ldcs(cur + i), p = __ldcs(prev + i);
+            if (kCopy) __stcs(prev + i, c);
+            float fn = 0.f, fd = 0.f;
+            rl1_acc(c, p, fn, fd);
+            num += fn;
+            den += fd;
+        }
+        // Elements past the last whole vector (fewer than kElems) go to thread 0 of block 0.
+        if (blockIdx.x == 0 && threadIdx.x == 0 && tail > 0) {
+            for (int t = 0; t < tail; ++t) {
+                float c, p;
+                if (kElems == 4) {
+                    c = static_cast<const float*>(cur_tail)[t];
+                    p = static_cast<const float*>(prev_tail)[t];
+                    if (kCopy) static_cast<float*>(prev_tail)[t] = c;
+                } else {
+                    const __nv_bfloat16 cb = static_cast<const __nv_bfloat16*>(cur_tail)[t];
+                    c = __bfloat162float(cb);
+                    p = __bfloat162float(static_cast<const __nv_bfloat16*>(prev_tail)[t]);
+                    if (kCopy) static_cast<__nv_bfloat16*>(prev_tail)[t] = cb;
+                }
+                num += fabsf(c - p);
+                den += fabsf(p);
+            }
+        }
+    }
+    rl1_block_sum2(num, den, sh);
+    if (threadIdx.x == 0) {
+        partials[blockIdx.x] = make_double2(num, den);
+        __threadfence();
+        const unsigned int t = atomicAdd(&ws->ticket, 1u);
+        is_last = (t == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    // Last block: fixed-order sum of the partials.
+    double a = 0.0, b = 0.0;
+    for (int k = threadIdx.x; k < static_cast<int>(gridDim.x); k += blockDim.x) {
+        const double2 v = __ldcg(&partials[k]);
+        a += v.x;
+        b += v.y;
+    }
+    __syncthreads();
+    rl1_block_sum2(a, b, sh);
+    if (threadIdx.x == 0) {
+        epi.finish(a, b, eval);
+        ws->ticket = 0u;
+    }
+}
+
+inline int rel_l1_blocks(int64_t nvec) {
+    const int64_t per = static_cast<int64_t>(kFbcThreads) * kFbcUnroll;
+    int64_t nb = (nvec + per - 1) / per;
+    if (nb < 1) nb = 1;
+    if (nb > kFbcMaxBlocks) nb = kFbcMaxBlocks;
+    return static_cast<int>(nb);
+}
+
+// Launch over n elements of dtype 0 (fp32) or 1 (bf16).  prev must be
+// writable when kCopy.
+template <bool kCopy, typename Epi>
+cudaError_t launch_rel_l1(const void* cur, const void* prev, int64_t n, int dtype, const Epi& epi, void* workspace,
+                          cudaStream_t stream) {
+    FbcWs* ws = static_cast<FbcWs*>(workspace);
+    void* pv = const_cast<void*>(prev);
+    if (dtype == 0) {
+        const int64_t nvec = n / 4;
+        const int tail = static_cast<int>(n - nvec * 4);
+        const float* c = static_cast<const float*>(cur);
+        float* p = static_cast<float*>(pv);
+        rel_l1_kernel<float4, 4, kCopy, Epi><<<rel_l1_blocks(nvec), kFbcThreads, 0, stream>>>(
+            reinterpret_cast<const float4*>(c), reinterpret_cast<float4*>(p), nvec, c + nvec * 4, p + nvec * 4,
+            tail, epi, ws);
+    } else {
+        const int64_t nvec = n / 8;
+        const int tail = static_cast<int>(n - nvec * 8);
+        const __nv_bfloat16* c = static_cast<const __nv_bfloat16*>(cur);
+        __nv_bfloat16* p = static_cast<__nv_bfloat16*>(pv);
+        rel_l1_kernel<uint4, 8, kCopy, Epi><<<rel_l1_blocks(nvec), kFbcThreads, 0, stream>>>(
+            reinterpret_cast<const uint4*>(c), reinterpret_cast<uint4*>(p), nvec, c + nvec * 8, p + nvec * 8, tail,
+            epi, ws);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ditk

@@ -170,6 +170,58 @@ def fbc_inputs(case: FbcCase):
     return cur.reshape(case.rows, case.cols), prev.reshape(case.rows, case.cols)
 
 
+@dataclass(frozen=True)
+class TrajectoryCase:
+    """A sequence of per-step tensors (first-block residuals or modulated
+    inputs) over the denoising steps of one generation: each step adds a
+    random drift whose size is drawn per step from [drift_lo, drift_hi]."""
+    name: str
+    rows: int
+    cols: int
+    dtype: str            # "f32" or "bf16"
+    steps: int
+    drift_lo: float
+    drift_hi: float
+    seed: int = 0
+
+    @property
+    def n(self) -> int:
+        return self.rows * self.cols
+
+
+# 28 steps (the FLUX.1-dev step count of the ParaAttention page) over a
+# 1024-token, 3072-wide residual; a ragged fp32 case; the long-video residual
+# width over 30 steps (the HunyuanVideo step count) at a reduced token count.
+TRAJ_IMAGE = TrajectoryCase("traj_flux28_1024x3072_bf16", 1024, 3072, "bf16", 28, 0.02, 0.2)
+TRAJ_RAGGED = TrajectoryCase("traj_ragged_999x37_f32", 999, 37, "f32", 24, 0.01, 0.3, seed=5)
+TRAJ_VIDEO = TrajectoryCase("traj_video30_4096x3072_bf16", 4096, 3072, "bf16", 30, 0.02, 0.15, seed=11)
+
+
+def trajectory(case: TrajectoryCase):
+    """List of ``steps`` arrays [rows, cols]: x_0 ~ N(0,1),
+    x_s = x_{s-1} + a_s * N(0,1) with a_s ~ U(drift_lo, drift_hi).
+
+    fp32 cases return float32 arrays; bf16 cases bf16 bit arrays (uint16),
+    each step formed in fp32 from the previous bf16 value and rounded once.
+    """
+    if case.dtype not in ("f32", "bf16"):
+        raise ValueError(f"unknown dtype {case.dtype}")
+    n = case.n
+    amp = _rng(case.seed, 7).uniform(case.drift_lo, case.drift_hi, size=case.steps).astype(np.float32)
+    out = []
+    x = _rng(case.seed, 8, 0).standard_normal(n, dtype=np.float32)
+    for s in range(case.steps):
+        if s > 0:
+            x = x + amp[s] * _rng(case.seed, 8, s).standard_normal(n, dtype=np.float32)
+        if case.dtype == "bf16":
+            b = bf16_bits(x)
+            x = bf16_to_f32(b)
+            out.append(b.reshape(case.rows, case.cols))
+        else:
+            out.append(x.reshape(case.rows, case.cols).copy())
+    return out
+
+
 def sample_rows(N: int, count: int, seed: int = 1) -> np.ndarray:
     """Sorted distinct query-row indices for sampled parity checks at full size.
 

@@ -181,6 +181,36 @@ dit_status fbc_rel_l1_noalloc(const void* r_cur, const void* r_prev, int64_t n, 
                               float threshold, double* out_rel, int32_t* out_skip, void* stream);
 
 /*
+ * dit_compare_stats — error of an output against a reference, per segment.
+ *
+ * Defined by: TMAP image-to-video blog, "keeping video quality": the error of
+ * each attention layer's 8-bit output over the denoising steps is what picks
+ * the layers that go back to 16-bit attention.  For each of n_segments
+ * contiguous segments of segment_len elements:
+ *   out[3s+0] = Σ|test − ref| / Σ|ref|              (relative L1)
+ *   out[3s+1] = Σ ref·test / sqrt(Σ ref² · Σ test²)  (cosine similarity)
+ *   out[3s+2] = max |test − ref|
+ * Empty norms: relative L1 is 0 when both sums are 0 and +inf when only Σ|ref|
+ * is; the cosine is 1 when both segments are all zero and 0 when one is.
+ *
+ *   ref, test   device arrays of n_segments * segment_len elements of
+ *               `dtype` (fp32 or bf16), aligned to the element size.  With
+ *               16-byte aligned bases and segments of whole 16-byte vectors
+ *               the kernel reads 16-byte vectors, else single elements.
+ *   n_segments  1..65535 (e.g. B*H for per-head errors of a [B,H,N,d] output).
+ *   out         device double[3 * n_segments].
+ *   workspace   device memory of dit_compare_workspace_bytes(...) bytes,
+ *               16-byte aligned, zero-filled before its first use; each call
+ *               leaves it zero-filled again.  Calls sharing it must be ordered.
+ *   Sums are fp32 over one 16-byte vector, fp64 beyond, in a fixed order:
+ *   deterministic for a given shape.
+ * Returns 0 from dit_compare_workspace_bytes for invalid shapes.
+ */
+size_t dit_compare_workspace_bytes(int64_t n_segments, int64_t segment_len, int dtype);
+dit_status dit_compare_stats(const void* ref, const void* test, int64_t n_segments, int64_t segment_len,
+                             int dtype, double* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * dit_get_device_status — synchronises `stream`, then returns and clears the
  * device-side error word of the current device (DIT_ERR_TIMEOUT if a bounded
  * wait inside a kernel ran out since the last call), or DIT_ERR_CUDA if the

@@ -153,3 +153,85 @@ def test_q8_quantize_argument_errors(lib):
     assert lib.dit_attn_q8_quantize(Q, K, V, 1, 2, 256, 64, None, 1, 0, WS, wsb, None) == dit.DIT_ERR_UNSUPPORTED
     assert lib.dit_attn_q8_quantize(Q, K, V, 1, 2, 256, 128, None, 1, 0, WS, 100, None) == dit.DIT_ERR_WORKSPACE
     assert lib.dit_attn_q8_quantize(0, K, V, 1, 2, 256, 128, None, 1, 0, WS, wsb, None) == dit.DIT_ERR_INVALID_ARG
+
+
+def test_cache_step_argument_errors(lib):
+    n = 4096
+    ws = lib.dit_cache_workspace_bytes(n)
+    assert ws == lib.fbc_rel_l1_workspace_bytes(n) and lib.dit_cache_workspace_bytes(0) == 0
+    pol = dit.dit_cache_policy()
+    ST, TR = 0x60000000, 0x61000000
+
+    def fb(**kw):
+        return lib.fbcache_step(kw.get("cur", Q), kw.get("prev", K), kw.get("n", n), kw.get("dtype", 1),
+                                kw.get("policy", ctypes.byref(pol)), kw.get("state", ST), kw.get("trace", TR),
+                                kw.get("cap", 8), kw.get("use_cond", 0), kw.get("cond", 0),
+                                kw.get("ws", O), kw.get("wsb", ws), None)
+    assert fb(cur=0) == dit.DIT_ERR_INVALID_ARG
+    assert fb(n=0) == dit.DIT_ERR_INVALID_ARG
+    assert fb(dtype=3) == dit.DIT_ERR_INVALID_ARG
+    assert fb(prev=K + 8) == dit.DIT_ERR_INVALID_ARG
+    assert fb(state=ST + 4) == dit.DIT_ERR_INVALID_ARG
+    assert fb(trace=TR + 4) == dit.DIT_ERR_INVALID_ARG
+    assert fb(cap=-1) == dit.DIT_ERR_INVALID_ARG
+    assert fb(policy=None) == dit.DIT_ERR_INVALID_ARG
+    assert fb(policy=ctypes.byref(dit.dit_cache_policy(max_warmup_steps=-1))) == dit.DIT_ERR_INVALID_ARG
+    assert fb(policy=ctypes.byref(dit.dit_cache_policy(residual_diff_threshold=float("inf")))) == \
+        dit.DIT_ERR_INVALID_ARG
+    assert fb(use_cond=2) == dit.DIT_ERR_INVALID_ARG
+    # a conditional handle that no capture on this stream created is refused
+    assert fb(use_cond=1, cond=12345) == dit.DIT_ERR_INVALID_ARG
+    assert fb(ws=0) == dit.DIT_ERR_WORKSPACE
+    assert fb(wsb=ws - 1) == dit.DIT_ERR_WORKSPACE
+
+    coeffs = (ctypes.c_double * 3)(0.0, 1.0, 0.0)
+
+    def tea(**kw):
+        return lib.teacache_step(kw.get("cur", Q), kw.get("prev", K), kw.get("n", n), kw.get("dtype", 1),
+                                 kw.get("coeffs", coeffs), kw.get("nc", 3), kw.get("thr", 0.1),
+                                 kw.get("state", ST), None, 0, kw.get("use_cond", 0), 0,
+                                 kw.get("ws", O), kw.get("wsb", ws), None)
+    assert tea(nc=0) == dit.DIT_ERR_INVALID_ARG
+    assert tea(nc=9) == dit.DIT_ERR_INVALID_ARG
+    assert tea(coeffs=None) == dit.DIT_ERR_INVALID_ARG
+    assert tea(coeffs=(ctypes.c_double * 3)(0.0, float("nan"), 0.0)) == dit.DIT_ERR_INVALID_ARG
+    assert tea(thr=float("nan")) == dit.DIT_ERR_INVALID_ARG
+    assert tea(prev=Q + 16) == dit.DIT_ERR_INVALID_ARG            # overlaps x_cur
+    assert tea(state=0) == dit.DIT_ERR_INVALID_ARG
+    assert tea(use_cond=1) == dit.DIT_ERR_INVALID_ARG
+    assert tea(wsb=0) == dit.DIT_ERR_WORKSPACE
+    assert lib.dit_cache_state_reset(None, None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.dit_cache_state_reset(ST + 4, None) == dit.DIT_ERR_INVALID_ARG
+
+
+def test_graph_plumbing_argument_errors(lib):
+    h = ctypes.c_ulonglong(0)
+    g = ctypes.c_void_p(0)
+    assert lib.dit_graph_capture_begin(None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.dit_graph_cond_create(None, ctypes.byref(h)) == dit.DIT_ERR_INVALID_ARG
+    assert lib.dit_graph_cond_body_begin(None, 0, None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.dit_graph_cond_body_begin(0x1000, 0, 0x1000) == dit.DIT_ERR_INVALID_ARG   # same stream
+    assert lib.dit_graph_cond_body_end(None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.dit_graph_capture_end(None, ctypes.byref(g)) == dit.DIT_ERR_INVALID_ARG
+    assert lib.dit_graph_launch(None, None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.dit_graph_destroy(None) == dit.DIT_ERR_INVALID_ARG
+
+
+def test_compare_argument_errors(lib):
+    assert lib.dit_compare_workspace_bytes(0, 10, 1) == 0
+    assert lib.dit_compare_workspace_bytes(65536, 10, 1) == 0
+    assert lib.dit_compare_workspace_bytes(4, 10, 9) == 0
+    ws = lib.dit_compare_workspace_bytes(4, 1000, 1)
+    assert ws >= 256 + 4 * 48
+
+    def cmp(**kw):
+        return lib.dit_compare_stats(kw.get("ref", Q), kw.get("test", K), kw.get("nseg", 4), kw.get("len", 1000),
+                                     kw.get("dtype", 1), kw.get("out", V), kw.get("ws", O), kw.get("wsb", ws), None)
+    assert cmp(ref=0) == dit.DIT_ERR_INVALID_ARG
+    assert cmp(nseg=0) == dit.DIT_ERR_INVALID_ARG
+    assert cmp(len=0) == dit.DIT_ERR_INVALID_ARG
+    assert cmp(dtype=2) == dit.DIT_ERR_INVALID_ARG
+    assert cmp(test=K + 1) == dit.DIT_ERR_INVALID_ARG                # not element aligned
+    assert cmp(out=V + 4) == dit.DIT_ERR_INVALID_ARG
+    assert cmp(ws=0) == dit.DIT_ERR_WORKSPACE
+    assert cmp(wsb=ws - 1) == dit.DIT_ERR_WORKSPACE
