@@ -272,21 +272,26 @@ def test_conditional_handle_of_another_capture_is_refused():
     y = torch.zeros_like(x)
     state = dit.cache_state()
     ws = dit.cache_workspace(64)
-    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    s1, s2, body = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     torch.cuda.synchronize()
-    dit.dit_graph_capture_begin(s1)
-    dit.dit_graph_capture_begin(s2)
-    try:
-        h1 = dit.dit_graph_cond_create(s1)
-        with pytest.raises(dit.DitError) as e:
-            dit.fbcache_step(x, y, dit.dit_cache_policy(), state, cond_handle=h1, workspace=ws, stream=s2)
-        assert e.value.status == dit.DIT_ERR_INVALID_ARG
-    finally:
-        g2 = dit.dit_graph_capture_end(s2)
-        g1 = dit.dit_graph_capture_end(s1)
-    for g in (g1, g2):
+    handles = {}
+
+    def step_fn(h):
+        handles["h1"] = h
+        # the same handle, offered to a step on another capturing stream
+        dit.dit_graph_capture_begin(s2)
+        try:
+            with pytest.raises(dit.DitError) as e:
+                dit.fbcache_step(x, y, dit.dit_cache_policy(), state, cond_handle=h, workspace=ws, stream=s2)
+            assert e.value.status == dit.DIT_ERR_INVALID_ARG
+        finally:
+            handles["g2"] = dit.dit_graph_capture_end(s2)
+        dit.fbcache_step(x, y, dit.dit_cache_policy(), state, cond_handle=h, workspace=ws, stream=s1)
+
+    g1 = _capture_step_graph(s1, body, step_fn, lambda: y.add_(1.0))
+    for g in (g1, handles["g2"]):
         dit.dit_graph_destroy(g)
-    # after the capture ended, the handle is refused outside any capture too
+    # after its capture ended, the handle is refused outside any capture too
     with pytest.raises(dit.DitError):
-        dit.fbcache_step(x, y, dit.dit_cache_policy(), state, cond_handle=h1, workspace=ws)
+        dit.fbcache_step(x, y, dit.dit_cache_policy(), state, cond_handle=handles["h1"], workspace=ws)
     torch.cuda.synchronize()
