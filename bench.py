@@ -233,6 +233,100 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- our arm
 
+def _time_calls(torch, stream, fn, reps):
+    """Mean device time (ms) of fn() over reps calls, CUDA events on `stream`."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    for _ in range(reps):
+        fn()
+    ev[1].record(stream)
+    ev[1].synchronize()
+    return ev[0].elapsed_time(ev[1]) / reps
+
+
+def measure_cache_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk, dv, case, reps):
+    """Device times (ms) of the step-cache calls and the output comparison on
+    the step's residual and outputs, and of one captured step graph whose
+    conditional body (the bf16 attention) is skipped or run."""
+    out = {}
+    n = dcur.numel()
+    ws = dit.cache_workspace(n, dev)
+    state = dit.cache_state(dev)
+    pol = dit.dit_cache_policy(max_warmup_steps=0, max_cached_steps=-1, max_continuous_cached_steps=-1,
+                               residual_diff_threshold=0.08)
+    dit.fbcache_step(dcur, dprev, pol, state, workspace=ws)  # step 0 stores; later steps evaluate
+    dit.fbcache_step(dcur, dprev, pol, state, workspace=ws)
+    out["fbcache_step_ms"] = _time_calls(torch, stream, lambda: dit.fbcache_step(dcur, dprev, pol, state,
+                                                                                 workspace=ws), reps)
+    xprev = torch.empty_like(dcur)
+    tstate = dit.cache_state(dev)
+    coeffs = [0.0, 1.0]
+    dit.teacache_step(dcur, xprev, coeffs, 0.3, tstate, workspace=ws)
+    out["teacache_step_ms"] = _time_calls(torch, stream, lambda: dit.teacache_step(dcur, xprev, coeffs, 0.3, tstate,
+                                                                                   workspace=ws), reps)
+    segs = case.B * case.H
+    cws = torch.zeros(dit.dit_compare_workspace_bytes(segs, do.numel() // segs, dit.DIT_DTYPE_BF16),
+                      dtype=torch.uint8, device=dev)
+    cout = torch.empty(segs, 3, dtype=torch.float64, device=dev)
+    dit.dit_compare_stats(do, do8, segs, out=cout, workspace=cws)
+    out["compare_ms"] = _time_calls(torch, stream, lambda: dit.dit_compare_stats(do, do8, segs, out=cout,
+                                                                                 workspace=cws), reps)
+    # One step graph: fbcache_step -> IF(compute) { bf16 attention }.  The
+    # residual compared with itself gives rel 0: with threshold 0.08 every
+    # step reuses the cache; with threshold 0 every step computes.
+    dgo = torch.empty_like(do)
+    body = torch.cuda.Stream(dev)
+    for name, thr in (("graph_cached_step_ms", 0.08), ("graph_computed_step_ms", 0.0)):
+        gpol = dit.dit_cache_policy(max_warmup_steps=0, max_cached_steps=-1, max_continuous_cached_steps=-1,
+                                    residual_diff_threshold=thr)
+        gstate = dit.cache_state(dev)
+        gs = torch.cuda.Stream(dev)
+        torch.cuda.synchronize(dev)
+        dit.dit_graph_capture_begin(gs)
+        body_open = False
+        try:
+            h = dit.dit_graph_cond_create(gs)
+            dit.fbcache_step(dcur, dcur, gpol, gstate, cond_handle=h, workspace=ws, stream=gs)
+            dit.dit_graph_cond_body_begin(gs, h, body)
+            body_open = True
+            dit.dit_attn_fwd(dq, dk, dv, o=dgo, stream=body)
+        finally:
+            if body_open:
+                dit.dit_graph_cond_body_end(body)
+            exe = dit.dit_graph_capture_end(gs)
+        try:
+            for _ in range(2):
+                dit.dit_graph_launch(exe, gs)
+            out[name] = _time_calls(torch, gs, lambda: dit.dit_graph_launch(exe, gs), max(3, reps // 2))
+            gs.synchronize()
+        finally:
+            dit.dit_graph_destroy(exe)
+        st = dit.read_cache_state(gstate)
+        expect = dit.DIT_CACHE_USE if thr > 0 else dit.DIT_CACHE_ABOVE_THRESHOLD
+        if st["last_decision"] != expect:
+            raise SystemExit(f"{name}: unexpected decision {st['last_decision']}")
+    return out
+
+
+def cache_rows_report(extra, fcase, case, peaks):
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    n = fcase.n
+    o_elems = case.B * case.H * case.N * case.d
+
+    def hbm_row(ms, nbytes, what):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": ms, "algorithmic_bytes": nbytes, "GB/s": gbs, "frac_of_measured_hbm": gbs / hbm, "what": what}
+
+    return {
+        "fbcache_step": hbm_row(extra["fbcache_step_ms"], 2 * n * 2, "read r_cur and r_prev (bf16)"),
+        "teacache_step": hbm_row(extra["teacache_step_ms"], 3 * n * 2, "read x_cur and x_prev, write x_prev"),
+        "compare_stats": hbm_row(extra["compare_ms"], 2 * o_elems * 2,
+                                 f"bf16 vs 8-bit attention output, {case.B * case.H} segments"),
+        "graph_step": {"cached_ms": extra["graph_cached_step_ms"], "computed_ms": extra["graph_computed_step_ms"],
+                       "what": "fbcache_step + IF node over one bf16 attention call; body skipped vs run"},
+    }
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -370,9 +464,14 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     prepass_ms = ep[0].elapsed_time(ep[1]) / K
 
+    # ---- the step caches and the output comparison (outside the timed step)
+    extra = measure_cache_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk, dv, case, K)
+
     # ---- max over ranks
-    ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms = max_over_ranks(
-        [ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms], dev, ws)
+    keys = sorted(extra)
+    vals = max_over_ranks([ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms] + [extra[k] for k in keys], dev, ws)
+    ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms = vals[:6]
+    extra = dict(zip(keys, vals[6:]))
 
     flops = 4.0 * case.B * case.H * case.N * case.N * case.d  # one attention call
     value = ws * K * 2 * flops / (ms * 1e-3) / 1e12
@@ -404,6 +503,7 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
+        "cache_rows": cache_rows_report(extra, fcase, case, peaks),
     }
     roof_bf16 = {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                  "frac": attn_tflops / peak,
