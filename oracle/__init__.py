@@ -49,6 +49,7 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         lib.oracle_attn_f64.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_double, _p, _i64]
         lib.oracle_attn_bf16in.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_double, _p, _i64]
+        lib.oracle_attn_lse_bf16in.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
         lib.oracle_fbc_rel_l1.argtypes = [_p, _p, _i64, ctypes.c_int, ctypes.c_double, _p, _p]
         lib.oracle_channel_mean.argtypes = [_p, _i64, _i64, _i64, _p]
         lib.oracle_quant_int8_blocks.argtypes = [_p, _i64, _i64, _i64, _i64, _p, _p, _p]
@@ -236,3 +237,44 @@ def compare_stats(ref, test, segments: int = 1):
             cos[s] = 1.0 if (xx == 0 and yy == 0) else 0.0
         mx[s] = np.abs(y - x).max() if x.size else 0.0
     return rel, cos, mx
+
+
+def attention_lse(q, k, v, scale: float | None = None):
+    """(O, lse) for bf16-bit inputs q [B,H,Nq,d], k and v [B,H,Nkv,d], in fp64.
+
+    lse[b,h,i] = ln sum_j exp(scale * q_i . k_j), the log-sum-exp of the row's
+    logits.  ParaAttention page, "Context Parallelism": the keys of one
+    attention may be split into chunks; these two results per chunk are what
+    ``merge_partials`` combines.
+    """
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    assert k.shape == (B, H, Nkv, d) and v.shape == k.shape
+    if scale is None:
+        scale = float(np.float32(1.0) / np.sqrt(np.float32(d)))
+    q, k, v = (np.ascontiguousarray(t, dtype=np.uint16) for t in (q, k, v))
+    out = np.empty((B, H, Nq, d), dtype=np.float64)
+    lse = np.empty((B, H, Nq), dtype=np.float64)
+    rc = _load().oracle_attn_lse_bf16in(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Nq, Nkv, d,
+                                        float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle attention failed ({rc})")
+    return out, lse
+
+
+def merge_partials(outs, lses):
+    """Attention over the union of key chunks from the per-chunk results, fp64.
+
+    With L_c the log-sum-exp of chunk c and O_c its normalised output:
+    L = ln sum_c exp(L_c) and O = sum_c exp(L_c - L) O_c (each chunk's
+    softmax denominator is exp(L_c); the union's is their sum).  The largest
+    L_c is subtracted before exponentiating.
+    outs: list of [..., d] arrays; lses: list of matching [...] arrays.
+    """
+    L = np.stack([np.asarray(x, dtype=np.float64) for x in lses])
+    O = np.stack([np.asarray(x, dtype=np.float64) for x in outs])
+    top = L.max(axis=0)
+    w = np.exp(L - top[None])
+    den = w.sum(axis=0)
+    out = (w[..., None] * O).sum(axis=0) / den[..., None]
+    return out, top + np.log(den)

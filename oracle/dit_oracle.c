@@ -72,9 +72,11 @@ int oracle_num_threads(void)
 #endif
 }
 
-/* One query row against all N keys of one head.  k, v: [N, d] fp64. */
-static void attn_row(const double *qrow, const double *k, const double *v,
-                     int64_t N, int64_t d, double scale, double *logit, double *orow)
+/* One query row against all N keys of one head.  k, v: [N, d] fp64.
+ * lse (may be NULL): ln sum_j exp(logit_j) = m + ln l. */
+static void attn_row_lse(const double *qrow, const double *k, const double *v,
+                         int64_t N, int64_t d, double scale, double *logit, double *orow,
+                         double *lse)
 {
     double m = -INFINITY;
     for (int64_t j = 0; j < N; ++j) {
@@ -96,6 +98,14 @@ static void attn_row(const double *qrow, const double *k, const double *v,
     }
     for (int64_t c = 0; c < d; ++c)
         orow[c] /= l;
+    if (lse)
+        *lse = m + log(l);
+}
+
+static void attn_row(const double *qrow, const double *k, const double *v,
+                     int64_t N, int64_t d, double scale, double *logit, double *orow)
+{
+    attn_row_lse(qrow, k, v, N, d, scale, logit, orow, NULL);
 }
 
 /* Attention over fp64 inputs q, k, v: [B, H, N, d] contiguous.
@@ -173,6 +183,51 @@ int oracle_attn_bf16in(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
 #pragma omp for schedule(dynamic, 1)
                 for (int64_t r = 0; r < nrows; ++r)
                     attn_row(qh + r * d, kh, vh, N, d, scale, logit, o + (bh * nrows + r) * d);
+                free(logit);
+            }
+        }
+    }
+    free(kh); free(vh); free(qh);
+    return fail ? 2 : 0;
+}
+
+/* Attention of Nq query rows against Nkv keys, with the log-sum-exp of every
+ * row: q [B, H, Nq, d], k and v [B, H, Nkv, d] as bf16 bits (widened exactly);
+ * o [B, H, Nq, d] and lse [B, H, Nq] fp64.  Context parallelism splits the keys
+ * of one attention into chunks ("ParaAttention", section "Context
+ * Parallelism"); the log-sum-exp of each chunk is what lets the chunk outputs
+ * be combined into the attention over all keys. */
+int oracle_attn_lse_bf16in(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o, double *lse,
+                           int64_t B, int64_t H, int64_t Nq, int64_t Nkv, int64_t d, double scale)
+{
+    if (Nq <= 0 || Nkv <= 0 || d <= 0)
+        return 1;
+    double *kh = (double *)malloc(sizeof(double) * (size_t)(Nkv * d));
+    double *vh = (double *)malloc(sizeof(double) * (size_t)(Nkv * d));
+    double *qh = (double *)malloc(sizeof(double) * (size_t)(Nq * d));
+    if (!kh || !vh || !qh) {
+        free(kh); free(vh); free(qh);
+        return 2;
+    }
+    int fail = 0;
+    for (int64_t bh = 0; bh < B * H && !fail; ++bh) {
+        for (int64_t e = 0; e < Nkv * d; ++e) {
+            kh[e] = bf16_to_double(k[bh * Nkv * d + e]);
+            vh[e] = bf16_to_double(v[bh * Nkv * d + e]);
+        }
+        for (int64_t e = 0; e < Nq * d; ++e)
+            qh[e] = bf16_to_double(q[bh * Nq * d + e]);
+#pragma omp parallel
+        {
+            double *logit = (double *)malloc(sizeof(double) * (size_t)Nkv);
+            if (!logit) {
+#pragma omp atomic write
+                fail = 1;
+            } else {
+#pragma omp for schedule(dynamic, 1)
+                for (int64_t r = 0; r < Nq; ++r)
+                    attn_row_lse(qh + r * d, kh, vh, Nkv, d, scale, logit, o + (bh * Nq + r) * d,
+                                 lse + bh * Nq + r);
                 free(logit);
             }
         }
