@@ -8,6 +8,8 @@ points raises.
 
 Entry points (same names as the C ABI in ``include/dit_attn.h``):
   * ``dit_attn_fwd(q, k, v, o=None, scale=None)``  — bf16 softmax attention
+  * ``dit_attn_fwd_ex(q, k, v, ..., lse=...)``      — Nq queries x Nkv keys, optional log-sum-exp
+  * ``dit_attn_merge(o_parts, lse_parts)``          — attention over the union of key chunks
   * ``dit_attn_fwd_q8(q, k, v, ...)``              — 8-bit attention (INT8 QKᵀ, FP8 or bf16 PV)
   * ``dit_attn_q8_quantize(q, k, v, ...)``         — its pre-pass alone
   * ``fbc_rel_l1(r_cur, r_prev, threshold, ...)``   — first-block-cache decision
@@ -47,6 +49,8 @@ _f = ctypes.c_float
 _sz = ctypes.c_size_t
 SIGNATURES = {
     "dit_attn_fwd": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p, _f, _p]),
+    "dit_attn_fwd_ex": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _f, _p]),
+    "dit_attn_merge": (_i, [_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
     "dit_attn_q8_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "dit_attn_fwd_q8": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p, _f, _i, _i, _p, _sz, _p]),
     "dit_attn_q8_quantize": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _i, _i, _p, _sz, _p]),
@@ -141,6 +145,70 @@ def dit_attn_fwd(q, k, v, o=None, scale: float | None = None, stream=None):
                           _attn_strides(q), float(scale) if scale else 0.0, _stream_ptr(stream))
     _check(st, "dit_attn_fwd")
     return o
+
+
+def dit_attn_fwd_ex(q, k, v, o=None, lse=None, scale: float | None = None, stream=None):
+    """Attention of q [B, H, Nq, d] against k, v [B, H, Nkv, d] (bf16 CUDA
+    tensors, unit stride in d; q and o share strides, k and v share theirs).
+
+    ``lse``: None (not computed), True (allocate), or an fp32 CUDA tensor
+    [B, H, Nq] to fill with each row's natural-log log-sum-exp.
+    Returns (o, lse or None)."""
+    import torch
+    lib = load_library()
+    if o is None:
+        o = torch.empty_like(q)
+    for t in (q, k, v, o):
+        if t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError("dit_attn_fwd_ex expects bf16 CUDA tensors")
+    if o.shape != q.shape or o.stride() != q.stride():
+        raise ValueError("q and o must share shape and strides")
+    if v.shape != k.shape or v.stride() != k.stride():
+        raise ValueError("k and v must share shape and strides")
+    B, H, Nq, d = q.shape
+    if k.shape[0] != B or k.shape[1] != H or k.shape[3] != d:
+        raise ValueError("k must be [B, H, Nkv, d] with q's B, H and d")
+    Nkv = k.shape[2]
+    if lse is True:
+        lse = torch.empty(B, H, Nq, dtype=torch.float32, device=q.device)
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous() or lse.numel() != B * H * Nq):
+        raise ValueError("lse must be a contiguous fp32 tensor of B*H*Nq elements")
+    st = lib.dit_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr() if lse is not None else None, B, H, Nq, Nkv, d,
+                             _attn_strides(q), _attn_strides(k), float(scale) if scale else 0.0, _stream_ptr(stream))
+    _check(st, "dit_attn_fwd_ex")
+    return o, lse
+
+
+def dit_attn_merge(o_parts, lse_parts, o=None, lse=None, stream=None):
+    """Merge per-key-chunk outputs (bf16 [B, H, N, d], equal strides) and their
+    log-sum-exps (fp32 [B, H, N]) into the attention over all chunks.
+    ``lse``: None, True (allocate) or an fp32 tensor.  Returns (o, lse or None)."""
+    import torch
+    lib = load_library()
+    n = len(o_parts)
+    if n != len(lse_parts) or n < 1:
+        raise ValueError("need as many log-sum-exps as outputs, at least one")
+    ref = o_parts[0]
+    for t in o_parts:
+        if t.dtype != torch.bfloat16 or t.shape != ref.shape or t.stride() != ref.stride():
+            raise ValueError("o_parts must be bf16 tensors of one shape and stride")
+    B, H, N, d = ref.shape
+    for t in lse_parts:
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.numel() != B * H * N:
+            raise ValueError("lse_parts must be contiguous fp32 tensors of B*H*N elements")
+    if o is None:
+        o = torch.empty_like(ref)
+    if o.shape != ref.shape or o.stride() != ref.stride():
+        raise ValueError("o must share the parts' shape and strides")
+    if lse is True:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=ref.device)
+    op = (ctypes.c_void_p * n)(*[t.data_ptr() for t in o_parts])
+    lp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in lse_parts])
+    st = lib.dit_attn_merge(op, lp, n, B, H, N, d, _attn_strides(ref), o.data_ptr(),
+                            lse.data_ptr() if lse is not None else None, _stream_ptr(stream))
+    _check(st, "dit_attn_merge")
+    return o, lse
 
 
 def _pv(pv_mode):

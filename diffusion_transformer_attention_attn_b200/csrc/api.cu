@@ -1,7 +1,7 @@
 // C ABI of libditattn.so (declared in include/dit_attn.h): argument
 // validation, TMA tensor-map encoding and launches.  Host code only; the
 // arithmetic of every call runs in the kernels of attn_bf16.cu, attn_q8.cu,
-// q8_prepass.cu and fbc_rel_l1.cu (the step caches and the output comparison
+// q8_prepass.cu, attn_merge.cu and fbc_rel_l1.cu (the step caches and the output comparison
 // have their own entry points in cache_step.cu and compare.cu).
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -135,6 +135,28 @@ dit_status encode_bf16_map(CUtensorMap* map, const void* base, int B, int H, int
 
 float default_scale(int d) { return 1.0f / std::sqrt(static_cast<float>(d)); }
 
+// (b, h, n) element strides of one bf16 [B, H, N, d] operand: given, or those
+// of the contiguous layout.  TMA needs every stride in bytes to be a multiple
+// of 16 below 2^40; rows must not alias (sn >= d).  span: bytes covered.
+dit_status resolve_strides(const int64_t* strides, int B, int H, int N, int d, int64_t* sb, int64_t* sh, int64_t* sn,
+                           int64_t* span) {
+    if (strides) {
+        *sb = strides[0];
+        *sh = strides[1];
+        *sn = strides[2];
+    } else {
+        *sn = d;
+        *sh = static_cast<int64_t>(N) * d;
+        *sb = static_cast<int64_t>(H) * N * d;
+    }
+    const int64_t st[3] = {*sb, *sh, *sn};
+    for (int i = 0; i < 3; ++i)
+        if (st[i] <= 0 || (st[i] * 2) % 16 != 0 || st[i] * 2 >= (int64_t(1) << 40)) return DIT_ERR_INVALID_ARG;
+    if (*sn < d) return DIT_ERR_INVALID_ARG;
+    *span = ((B - 1) * *sb + (H - 1) * *sh + (N - 1) * *sn + d) * 2;
+    return DIT_OK;
+}
+
 // 4-D map {128 B, N, H, B} over contiguous 8-bit codes [B, H, N, 128] inside
 // the workspace, box {128, 128, 1, 1}, 128-B swizzle.
 dit_status encode_u8_map(CUtensorMap* map, const void* base, int B, int H, int N) {
@@ -174,6 +196,75 @@ using namespace ditk;
 
 extern "C" {
 
+dit_status dit_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                           int Nkv, int d, const int64_t* q_strides, const int64_t* kv_strides, float scale,
+                           void* stream) {
+    if (!q || !k || !v || !o) return DIT_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || Nq < 1 || Nkv < 1 || d < 1) return DIT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DIT_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return DIT_ERR_UNSUPPORTED;
+    if (Nq > (1 << 30) || Nkv > (1 << 30) || static_cast<int64_t>(B) * H > (1 << 24)) return DIT_ERR_UNSUPPORTED;
+    int64_t qb, qh, qn, kb, kh, kn, qspan, kspan;
+    dit_status st = resolve_strides(q_strides, B, H, Nq, d, &qb, &qh, &qn, &qspan);
+    if (st != DIT_OK) return st;
+    if ((st = resolve_strides(kv_strides, B, H, Nkv, d, &kb, &kh, &kn, &kspan)) != DIT_OK) return st;
+    const uintptr_t uo = reinterpret_cast<uintptr_t>(o);
+    auto hit = [](uintptr_t a, int64_t sa, const void* p, int64_t sp) {
+        const uintptr_t b = reinterpret_cast<uintptr_t>(p);
+        return a < b + static_cast<uintptr_t>(sp) && b < a + static_cast<uintptr_t>(sa);
+    };
+    if (hit(uo, qspan, q, qspan) || hit(uo, qspan, k, kspan) || hit(uo, qspan, v, kspan)) return DIT_ERR_INVALID_ARG;
+    if (lse) {
+        if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return DIT_ERR_INVALID_ARG;
+        const int64_t lspan = static_cast<int64_t>(B) * H * Nq * 4;
+        const uintptr_t ul = reinterpret_cast<uintptr_t>(lse);
+        if (hit(ul, lspan, o, qspan) || hit(ul, lspan, q, qspan) || hit(ul, lspan, k, kspan) ||
+            hit(ul, lspan, v, kspan))
+            return DIT_ERR_INVALID_ARG;
+    }
+    if (!(scale == scale) || std::isinf(scale)) return DIT_ERR_INVALID_ARG;
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    CUtensorMap tq, tk, tv;
+    if ((st = encode_bf16_map(&tq, q, B, H, Nq, d, qb, qh, qn)) != DIT_OK) return st;
+    if ((st = encode_bf16_map(&tk, k, B, H, Nkv, d, kb, kh, kn)) != DIT_OK) return st;
+    if ((st = encode_bf16_map(&tv, v, B, H, Nkv, d, kb, kh, kn)) != DIT_OK) return st;
+    const float s = scale > 0.f ? scale : default_scale(d);
+    const float scale_log2 = static_cast<float>(static_cast<double>(s) * 1.4426950408889634);
+    cudaError_t e = launch_attn_bf16(tq, tk, tv, o, qb, qh, qn, B, H, Nq, Nkv, d, scale_log2, lse, ds->err_word,
+                                     static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+dit_status dit_attn_merge(const void* const* o_parts, const float* const* lse_parts, int n_parts, int B, int H, int N,
+                          int d, const int64_t* strides, void* o, float* lse, void* stream) {
+    if (!o_parts || !lse_parts || !o || n_parts < 1 || n_parts > kMaxMergeParts) return DIT_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || N < 1 || d < 8 || d > 256 || d % 8 != 0) return DIT_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * H * N > (int64_t(1) << 36)) return DIT_ERR_UNSUPPORTED;
+    int64_t sb, sh, sn, span;
+    dit_status st = resolve_strides(strides, B, H, N, d, &sb, &sh, &sn, &span);
+    if (st != DIT_OK) return st;
+    if (!aligned16(o)) return DIT_ERR_INVALID_ARG;
+    const int64_t lspan = static_cast<int64_t>(B) * H * N * 4;
+    auto hit = [](const void* a, int64_t sa, const void* p, int64_t sp) {
+        const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(p);
+        return x < y + static_cast<uintptr_t>(sp) && y < x + static_cast<uintptr_t>(sa);
+    };
+    for (int c = 0; c < n_parts; ++c) {
+        if (!o_parts[c] || !lse_parts[c] || !aligned16(o_parts[c])) return DIT_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(lse_parts[c]) & 3u) != 0) return DIT_ERR_INVALID_ARG;
+        // the output may not overwrite an input still to be read
+        if (hit(o, span, o_parts[c], span) || hit(o, span, lse_parts[c], lspan)) return DIT_ERR_INVALID_ARG;
+        if (lse && (hit(lse, lspan, o_parts[c], span) || hit(lse, lspan, lse_parts[c], lspan)))
+            return DIT_ERR_INVALID_ARG;
+    }
+    if (lse && ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || hit(lse, lspan, o, span))) return DIT_ERR_INVALID_ARG;
+    if (!device_state(&st)) return st;
+    cudaError_t e = launch_attn_merge(o_parts, lse_parts, n_parts, B, H, N, d, sb, sh, sn, o, lse,
+                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
 dit_status dit_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
                         const int64_t* strides, float scale, void* stream) {
     int64_t sb, sh, sn;
@@ -188,7 +279,7 @@ dit_status dit_attn_fwd(const void* q, const void* k, const void* v, void* o, in
     if ((st = encode_bf16_map(&tv, v, B, H, N, d, sb, sh, sn)) != DIT_OK) return st;
     const float s = scale > 0.f ? scale : default_scale(d);
     const float scale_log2 = static_cast<float>(static_cast<double>(s) * 1.4426950408889634);
-    cudaError_t e = launch_attn_bf16(tq, tk, tv, o, sb, sh, sn, B, H, N, d, scale_log2, ds->err_word,
+    cudaError_t e = launch_attn_bf16(tq, tk, tv, o, sb, sh, sn, B, H, N, N, d, scale_log2, nullptr, ds->err_word,
                                      static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }

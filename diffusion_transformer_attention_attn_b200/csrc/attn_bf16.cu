@@ -29,6 +29,12 @@
 // and the row sum l with it.  P = 2^(t - m) ≤ 256 is exact enough in bf16
 // and O, l are fp32.  Keys at or past N (the ragged last tile, zero-filled
 // by TMA) get t = -inf, hence P = 0.
+//
+// Queries and keys may have different lengths (Nq rows against Nkv keys), so
+// one launch can cover one chunk of a longer key sequence.  With `lse` given,
+// each row also stores its log-sum-exp, ln Σ_j exp(scale·s_j) =
+// ln 2 · (m + log2 l), the quantity that lets the outputs of several key
+// chunks be merged into the attention over all of them (dit_attn_merge).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -118,7 +124,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                          const __grid_constant__ CUtensorMap tv, __nv_bfloat16* __restrict__ o, int64_t sb,
-                         int64_t sh, int64_t sn, int H, int N, int n_pairs, float scale_log2, int* err) {
+                         int64_t sh, int64_t sn, int H, int Nq, int Nkv, int n_pairs, float scale_log2,
+                         float* __restrict__ lse, int* err) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -134,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int b = bh / H;
     const int h = bh % H;
     const int q0 = pair * 2 * kBM;
-    const int nkv = (N + kBN - 1) / kBN;
+    const int nkv = (Nkv + kBN - 1) / kBN;
 
     if (threadIdx.x == 0) {
         mbar_init(bars.q_full, 1);
@@ -313,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             uint32_t r[kBN / 32][32];
             auto X = [&](int col) { return __uint_as_float(r[col >> 5][col & 31]); };
-            const int valid = N - j * kBN;  // keys of this tile below N
+            const int valid = Nkv - j * kBN;  // keys of this tile below Nkv
             // Row max over the tile; keys past N are left out.  Full tiles load
             // S in 32-column chunks and fold each chunk into 8 independent
             // 3-input max chains while the next chunk is in flight.
@@ -429,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 lsum = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
             l += lsum.x + lsum.y;
         }
-        // Epilogue: O / l -> bf16 -> global (rows at or past N are padding).
+        // Epilogue: O / l -> bf16 -> global (rows at or past Nq are padding).
         if (ok) ok = mbar_wait(&bars.o_ready[wg], (nkv - 1) & 1, abort_flag, err);
         if (ok) {
             tc_fence_after();
@@ -446,13 +453,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-                if (qrow < N) {
+                if (qrow < Nq) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                 }
             }
+            if (lse != nullptr && qrow < Nq)
+                lse[static_cast<int64_t>(bh) * Nq + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
         }
     }
 
@@ -466,7 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int64_t sb,
-                     int64_t sh, int64_t sn, int B, int H, int N, float scale_log2, int* err, cudaStream_t stream) {
+                     int64_t sh, int64_t sn, int B, int H, int Nq, int Nkv, float scale_log2, float* lse, int* err,
+                     cudaStream_t stream) {
     using C = Cfg<D>;
     static_assert(C::kSmemBytes <= 232448, "shared memory budget");
     // The register split inside the kernel needs the full launch allotment.
@@ -477,22 +487,22 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
     e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const int n_qt = (N + kBM - 1) / kBM;
+    const int n_qt = (Nq + kBM - 1) / kBM;
     const int n_pairs = (n_qt + 1) / 2;
     const int64_t grid = static_cast<int64_t>(B) * H * n_pairs;
     if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
     attn_fwd_bf16_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(
-        tq, tk, tv, static_cast<__nv_bfloat16*>(o), sb, sh, sn, H, N, n_pairs, scale_log2, err);
+        tq, tk, tv, static_cast<__nv_bfloat16*>(o), sb, sh, sn, H, Nq, Nkv, n_pairs, scale_log2, lse, err);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                             int64_t sb, int64_t sh, int64_t sn, int B, int H, int N, int d, float scale_log2,
-                             int* err, cudaStream_t stream) {
-    if (d == 128) return launch_d<128>(tq, tk, tv, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
-    if (d == 64) return launch_d<64>(tq, tk, tv, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
+                             int64_t sb, int64_t sh, int64_t sn, int B, int H, int Nq, int Nkv, int d,
+                             float scale_log2, float* lse, int* err, cudaStream_t stream) {
+    if (d == 128) return launch_d<128>(tq, tk, tv, o, sb, sh, sn, B, H, Nq, Nkv, scale_log2, lse, err, stream);
+    if (d == 64) return launch_d<64>(tq, tk, tv, o, sb, sh, sn, B, H, Nq, Nkv, scale_log2, lse, err, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -12,9 +12,17 @@ namespace ditk {
 // Softmax attention, bf16 in/out.  tq/tk/tv: 4-D tensor maps {d, N, H, B} with
 // a {64, 128, 1, 1} box and 128-byte swizzle.  o: output base; s*: element
 // strides of (b, h, n).  scale_log2 = scale * log2(e).  err: device error word.
+// Nq query rows attend to Nkv keys (tq has Nq rows, tk/tv Nkv).  lse: NULL or
+// fp32 [B, H, Nq] contiguous, the natural-log log-sum-exp of each row.
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                             int64_t sb, int64_t sh, int64_t sn, int B, int H, int N, int d, float scale_log2,
-                             int* err, cudaStream_t stream);
+                             int64_t sb, int64_t sh, int64_t sn, int B, int H, int Nq, int Nkv, int d,
+                             float scale_log2, float* lse, int* err, cudaStream_t stream);
+
+// Merge of per-key-chunk outputs (see dit_attn_merge in dit_attn.h).
+constexpr int kMaxMergeParts = 16;
+cudaError_t launch_attn_merge(const void* const* o_parts, const float* const* lse_parts, int n_parts, int B, int H,
+                              int N, int d, int64_t sb, int64_t sh, int64_t sn, void* o, float* lse,
+                              cudaStream_t stream);
 
 // ---- 8-bit path (d = 128) ----------------------------------------------
 // Tokens per statistics chunk of the pre-pass.

@@ -72,6 +72,48 @@ dit_status dit_attn_fwd(const void* q, const void* k, const void* v, void* o,
                         float scale, void* stream);
 
 /*
+ * dit_attn_fwd_ex — dit_attn_fwd with separate query and key lengths and an
+ * optional log-sum-exp output: Nq query rows attend to Nkv keys, and
+ *   lse[b,h,i] = ln Σ_j exp(scale · q_i·k_j)        (fp32, natural log)
+ *
+ * Defined by: "ParaAttention" (diffusers docs), section "Context Parallelism",
+ * and the TMAP image-to-video blog, section on sequence parallelism: the keys
+ * of one attention may be split into chunks (one per device in ring-style
+ * context parallelism).  Each chunk's normalised output and log-sum-exp are
+ * what dit_attn_merge combines into the attention over all keys.
+ *
+ *   q, o        bf16 [B, H, Nq, d], strides q_strides (elements; NULL:
+ *               contiguous); o must not overlap any input.
+ *   k, v        bf16 [B, H, Nkv, d], strides kv_strides (NULL: contiguous).
+ *               A chunk of a longer K/V is addressed by offsetting the base
+ *               pointers by (start · sn) elements and passing its length.
+ *   lse         device fp32 [B, H, Nq] contiguous, or NULL.
+ *   Nq, Nkv >= 1; d in {64, 128}; alignment and stride rules as dit_attn_fwd.
+ */
+dit_status dit_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int H, int Nq, int Nkv, int d,
+                           const int64_t* q_strides, const int64_t* kv_strides,
+                           float scale, void* stream);
+
+/*
+ * dit_attn_merge — the attention over the union of key chunks, from the
+ * chunks' outputs and log-sum-exps:
+ *   lse = ln Σ_c exp(lse_c),   o = Σ_c exp(lse_c − lse) · o_c
+ * (same passages as dit_attn_fwd_ex).
+ *
+ *   o_parts     host array of n_parts (1..16) device pointers, bf16
+ *               [B, H, N, d] with `strides` (NULL: contiguous), 16-byte aligned.
+ *   lse_parts   host array of n_parts device pointers, fp32 [B, H, N].
+ *   o           bf16 output with the same strides; lse: fp32 [B, H, N] or NULL.
+ *               Neither may overlap an input.
+ *   d a multiple of 8 up to 256.  A row whose every lse_c is −inf gets o = 0
+ *   and lse = −inf.  Weights use the largest lse_c as the shift (fp32).
+ */
+dit_status dit_attn_merge(const void* const* o_parts, const float* const* lse_parts, int n_parts,
+                          int B, int H, int N, int d, const int64_t* strides,
+                          void* o, float* lse, void* stream);
+
+/*
  * dit_attn_fwd_q8 — the same attention with 8-bit operands.
  *
  * Defined by: "TMAP image-to-video inference acceleration" (joto.ai), section

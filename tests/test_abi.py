@@ -235,3 +235,38 @@ def test_compare_argument_errors(lib):
     assert cmp(out=V + 4) == dit.DIT_ERR_INVALID_ARG
     assert cmp(ws=0) == dit.DIT_ERR_WORKSPACE
     assert cmp(wsb=ws - 1) == dit.DIT_ERR_WORKSPACE
+
+
+def test_attn_ex_and_merge_argument_errors(lib):
+    def ex(**kw):
+        qs = kw.get("qs")
+        ks = kw.get("ks")
+        return lib.dit_attn_fwd_ex(kw.get("q", Q), kw.get("k", K), kw.get("v", V), kw.get("o", O), kw.get("lse", None),
+                                   1, 2, kw.get("Nq", 256), kw.get("Nkv", 512), kw.get("d", 64),
+                                   (ctypes.c_int64 * 3)(*qs) if qs else None,
+                                   (ctypes.c_int64 * 3)(*ks) if ks else None, kw.get("scale", 0.0), None)
+    assert ex(Nq=0) == dit.DIT_ERR_INVALID_ARG
+    assert ex(Nkv=0) == dit.DIT_ERR_INVALID_ARG
+    assert ex(d=96) == dit.DIT_ERR_UNSUPPORTED
+    assert ex(o=0) == dit.DIT_ERR_INVALID_ARG
+    assert ex(v=V + 8) == dit.DIT_ERR_INVALID_ARG
+    assert ex(o=K + 1024) == dit.DIT_ERR_INVALID_ARG               # inside k
+    assert ex(lse=O + 2) == dit.DIT_ERR_INVALID_ARG                # misaligned
+    assert ex(lse=O + 64) == dit.DIT_ERR_INVALID_ARG               # overlaps o
+    assert ex(ks=(512 * 64 * 2, 512 * 64, 60)) == dit.DIT_ERR_INVALID_ARG
+    assert ex(scale=float("inf")) == dit.DIT_ERR_INVALID_ARG
+
+    def merge(n=2, parts=None, lparts=None, o=0x70000000, lse=None, N=256, d=64):
+        parts = parts or [Q, K][:n] + [V] * max(0, n - 2)
+        lparts = lparts or [0x71000000 + 0x100000 * i for i in range(n)]
+        op = (ctypes.c_void_p * max(n, 1))(*parts[:max(n, 1)])
+        lp = (ctypes.c_void_p * max(n, 1))(*lparts[:max(n, 1)])
+        return lib.dit_attn_merge(op, lp, n, 1, 2, N, d, None, o, lse, None)
+    assert merge(n=0) == dit.DIT_ERR_INVALID_ARG
+    assert merge(n=17) == dit.DIT_ERR_INVALID_ARG
+    assert merge(d=12) == dit.DIT_ERR_INVALID_ARG
+    assert merge(o=0x70000008) == dit.DIT_ERR_INVALID_ARG           # misaligned output
+    assert merge(parts=[Q + 8, K]) == dit.DIT_ERR_INVALID_ARG       # misaligned part
+    assert merge(lparts=[0x71000002, 0x71100000]) == dit.DIT_ERR_INVALID_ARG
+    assert merge(o=Q) == dit.DIT_ERR_INVALID_ARG                    # output overwrites a part
+    assert merge(lse=0x71000000) == dit.DIT_ERR_INVALID_ARG         # lse overwrites a part's lse

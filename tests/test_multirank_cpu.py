@@ -42,7 +42,7 @@ def test_two_gloo_ranks_max_time_and_distinct_replicas():
     import torch.multiprocessing as mp
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         results = mgr.dict()
         mp.spawn(_worker, args=(world, port, results), nprocs=world, join=True)
         res = dict(results)
