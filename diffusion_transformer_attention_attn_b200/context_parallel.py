@@ -1,0 +1,131 @@
+"""Context parallelism for the attention call: one process per GPU, the token
+sequence split evenly across the ranks of a ``torch.distributed`` group.
+
+Two schemes, both from "ParaAttention" (diffusers docs), section "Context
+Parallelism", and the TMAP image-to-video blog, section on sequence
+parallelism (Ulysses, with its all-to-all overlapped with the surrounding
+work):
+
+* ``ulysses_attention`` — each rank holds all heads of its N/P tokens.  One
+  all-to-all regroups Q, K and V so that each rank holds H/P heads of all N
+  tokens; attention runs locally per head (the DiT attention has no mask and
+  heads are independent); a second all-to-all returns each rank's tokens.
+* ``ring_attention`` — each rank keeps its queries and passes its K/V chunk
+  around the ring; every step attends the local queries to the chunk in hand
+  (``dit_attn_fwd_ex`` with log-sum-exp), while the next chunk is already in
+  flight, and the per-chunk results are merged (``dit_attn_merge``).
+
+The collectives are torch.distributed calls (NCCL between GPUs); the attention
+and the merge are the library's kernels.  ``attn_fn`` / ``attn_lse_fn`` /
+``merge_fn`` may be replaced, e.g. to run the data movement on CPU ranks.
+"""
+from __future__ import annotations
+
+
+def _group_info(group):
+    import torch.distributed as dist
+    return dist.get_world_size(group), dist.get_rank(group)
+
+
+def _default_attn(q, k, v):
+    from . import dit_attn_fwd
+    return dit_attn_fwd(q, k, v)
+
+
+def _default_attn_lse(q, k, v):
+    from . import dit_attn_fwd_ex
+    return dit_attn_fwd_ex(q, k, v, lse=True)
+
+
+def _default_merge(outs, lses):
+    from . import dit_attn_merge
+    return dit_attn_merge(outs, lses, lse=True)
+
+
+def seq_to_heads(xs, world: int, group=None):
+    """All-to-all of sequence-sharded tensors to head-sharded ones.
+
+    xs: list of [B, H, Nl, d] tensors (this rank's Nl = N/P tokens, all heads),
+    H divisible by the group size P.  Returns [B, H/P, P*Nl, d] tensors: head
+    group r of this rank r, tokens in global order (rank-major).  All tensors
+    travel in one all-to-all.
+    """
+    import torch
+    import torch.distributed as dist
+    B, H, Nl, d = xs[0].shape
+    P = world
+    hp = H // P
+    # [P (destination head group), T, B, H/P, Nl, d]
+    send = torch.stack([x.reshape(B, P, hp, Nl, d) for x in xs], dim=0).permute(2, 0, 1, 3, 4, 5).contiguous()
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    # recv[src] = src's tokens of my heads -> [T, B, H/P, P*Nl, d]
+    out = recv.permute(1, 2, 3, 0, 4, 5).reshape(len(xs), B, hp, P * Nl, d)
+    return [out[i] for i in range(len(xs))]
+
+
+def heads_to_seq(y, world: int, group=None):
+    """Inverse of ``seq_to_heads`` for one tensor: [B, H/P, P*Nl, d] ->
+    [B, H, Nl, d] (this rank's tokens, all heads, head groups rank-major)."""
+    import torch
+    import torch.distributed as dist
+    B, hp, N, d = y.shape
+    P = world
+    Nl = N // P
+    send = y.reshape(B, hp, P, Nl, d).permute(2, 0, 1, 3, 4).contiguous()   # [P (token owner), B, H/P, Nl, d]
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    return recv.permute(1, 0, 2, 3, 4).reshape(B, P * hp, Nl, d)
+
+
+def ulysses_attention(q, k, v, group=None, attn_fn=None):
+    """Attention over the full sequence from sequence-sharded [B, H, N/P, d]
+    q, k, v; returns this rank's [B, H, N/P, d] output."""
+    world, _ = _group_info(group)
+    B, H, Nl, d = q.shape
+    if H % world:
+        raise ValueError(f"{H} heads do not split over {world} ranks")
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share their shape")
+    attn = attn_fn or _default_attn
+    if world == 1:
+        return attn(q, k, v)
+    qh, kh, vh = seq_to_heads([q, k, v], world, group)
+    return heads_to_seq(attn(qh, kh, vh), world, group)
+
+
+def ring_attention(q, k, v, group=None, attn_lse_fn=None, merge_fn=None):
+    """Attention of this rank's queries [B, H, Nl, d] to all ranks' keys, the
+    K/V chunks travelling around the ring (rank r sends to r+1 and receives
+    from r-1).  Returns (o, lse) for the local queries."""
+    import torch
+    import torch.distributed as dist
+    world, rank = _group_info(group)
+    attn = attn_lse_fn or _default_attn_lse
+    merge = merge_fn or _default_merge
+    kv = torch.stack([k, v], dim=0).contiguous()
+    outs, lses = [], []
+    nxt = (rank + 1) % world
+    prv = (rank - 1) % world
+    for step in range(world):
+        reqs = []
+        if step + 1 < world:
+            buf = torch.empty_like(kv)
+            g_nxt = dist.get_global_rank(group, nxt) if group is not None else nxt
+            g_prv = dist.get_global_rank(group, prv) if group is not None else prv
+            ops = [dist.P2POp(dist.isend, kv, g_nxt, group), dist.P2POp(dist.irecv, buf, g_prv, group)]
+            reqs = dist.batch_isend_irecv(ops)
+        o_c, l_c = attn(q, kv[0], kv[1])
+        outs.append(o_c)
+        lses.append(l_c)
+        for r in reqs:
+            r.wait()
+        if step + 1 < world:
+            kv = buf
+        # Merge as the parts arrive once the merge kernel's fan-in is reached.
+        if len(outs) == 16:
+            o_m, l_m = merge(outs, lses)
+            outs, lses = [o_m], [l_m]
+    if len(outs) == 1:
+        return outs[0], lses[0]
+    return merge(outs, lses)

@@ -1,0 +1,117 @@
+"""The data movement of the context-parallel attention on CPU ranks (gloo).
+
+Each rank holds N/P tokens of Q, K and V.  With the oracle's fp64 attention
+standing in for the kernel (injected through the attn_fn / attn_lse_fn /
+merge_fn arguments), Ulysses must reproduce the full-sequence attention
+exactly (every head sees the same keys in the same order) and the ring must
+match it to fp64 rounding (chunks merged through their log-sum-exps).
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _global_inputs(B, H, N, d, seed=0):
+    from diffusion_transformer_attention_attn_b200 import inputs
+    return inputs.attn_inputs(inputs.AttnCase("cp", B, H, N, d, seed=seed))
+
+
+def _worker(rank, world, port, scheme, shape, results):
+    import torch.distributed as dist
+
+    import oracle
+    from diffusion_transformer_attention_attn_b200 import context_parallel as cp
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, H, N, d = shape
+        q, k, v = _global_inputs(B, H, N, d)
+        Nl = N // world
+        sl = slice(rank * Nl, (rank + 1) * Nl)
+        # bf16 values travel widened to fp32 (exact); gloo has no 16-bit all-to-all
+        from diffusion_transformer_attention_attn_b200 import inputs
+        tq, tk, tv = (torch.from_numpy(inputs.bf16_to_f32(np.ascontiguousarray(x[:, :, sl]))) for x in (q, k, v))
+
+        def bits(t):
+            return inputs.bf16_bits(t.contiguous().numpy())
+
+        if scheme == "ulysses":
+            def attn(a, b, c):
+                return torch.from_numpy(oracle.attention(bits(a), bits(b), bits(c)))
+            out = cp.ulysses_attention(tq, tk, tv, attn_fn=attn)
+            results[rank] = out.numpy()
+        else:
+            def attn_lse(a, b, c):
+                o, l = oracle.attention_lse(bits(a), bits(b), bits(c))
+                return torch.from_numpy(o), torch.from_numpy(l)
+
+            def merge(outs, lses):
+                o, l = oracle.merge_partials([x.numpy() for x in outs], [x.numpy() for x in lses])
+                return torch.from_numpy(o), torch.from_numpy(l)
+            o, l = cp.ring_attention(tq, tk, tv, attn_lse_fn=attn_lse, merge_fn=merge)
+            results[rank] = (o.numpy(), l.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(scheme, world, shape):
+    import torch.multiprocessing as mp
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_worker, args=(world, port, scheme, shape, results), nprocs=world, join=True,
+                           start_method="spawn")
+        return dict(results)
+
+
+@pytest.mark.parametrize("world,shape", [(2, (1, 4, 96, 16)), (4, (2, 8, 64, 32))])
+def test_ulysses_matches_full_attention_exactly(world, shape):
+    import oracle
+    B, H, N, d = shape
+    q, k, v = _global_inputs(B, H, N, d)
+    ref = oracle.attention(q, k, v)
+    res = _run("ulysses", world, shape)
+    got = np.concatenate([res[r] for r in range(world)], axis=2)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("world,shape", [(2, (1, 2, 96, 16)), (4, (1, 3, 128, 8))])
+def test_ring_matches_full_attention(world, shape):
+    import oracle
+    B, H, N, d = shape
+    q, k, v = _global_inputs(B, H, N, d)
+    ref, ref_lse = oracle.attention_lse(q, k, v)
+    res = _run("ring", world, shape)
+    got = np.concatenate([res[r][0] for r in range(world)], axis=2)
+    lse = np.concatenate([res[r][1] for r in range(world)], axis=2)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def test_world_of_one_runs_locally():
+    from diffusion_transformer_attention_attn_b200 import context_parallel as cp
+    import torch.distributed as dist
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised")
+    store = dist.HashStore()
+    dist.init_process_group("gloo", store=store, rank=0, world_size=1)
+    try:
+        x = torch.zeros(1, 3, 4, 8)
+        # world 1: the attention runs locally, no collective
+        out = cp.ulysses_attention(x, x, x, attn_fn=lambda a, b, c: a + 1)
+        assert torch.equal(out, x + 1)
+    finally:
+        dist.destroy_process_group()
