@@ -244,10 +244,14 @@ def _time_calls(torch, stream, fn, reps):
     return ev[0].elapsed_time(ev[1]) / reps
 
 
-def measure_cache_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk, dv, case, reps):
+CHUNKS = 4  # key chunks of the one-GPU ring emulation
+
+
+def measure_next_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk, dv, case, reps):
     """Device times (ms) of the step-cache calls and the output comparison on
-    the step's residual and outputs, and of one captured step graph whose
-    conditional body (the bf16 attention) is skipped or run."""
+    the step's residual and outputs, of one captured step graph whose
+    conditional body (the bf16 attention) is skipped or run, and of the
+    key-chunked attention (CHUNKS chunks with log-sum-exp, then the merge)."""
     out = {}
     n = dcur.numel()
     ws = dit.cache_workspace(n, dev)
@@ -305,10 +309,31 @@ def measure_cache_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk, dv
         expect = dit.DIT_CACHE_USE if thr > 0 else dit.DIT_CACHE_ABOVE_THRESHOLD
         if st["last_decision"] != expect:
             raise SystemExit(f"{name}: unexpected decision {st['last_decision']}")
+    # Key-chunked attention: CHUNKS calls of dit_attn_fwd_ex on K/V views, then the merge.
+    N = case.N
+    bounds = [N * c // CHUNKS for c in range(CHUNKS + 1)]
+    parts = [(torch.empty_like(dq), torch.empty(case.B, case.H, N, dtype=torch.float32, device=dev))
+             for _ in range(CHUNKS)]
+    mo = torch.empty_like(dq)
+    ml = torch.empty(case.B, case.H, N, dtype=torch.float32, device=dev)
+
+    def chunked():
+        for c in range(CHUNKS):
+            a, b = bounds[c], bounds[c + 1]
+            dit.dit_attn_fwd_ex(dq, dk[:, :, a:b], dv[:, :, a:b], o=parts[c][0], lse=parts[c][1])
+
+    def merge():
+        dit.dit_attn_merge([p[0] for p in parts], [p[1] for p in parts], o=mo, lse=ml)
+
+    chunked()
+    merge()
+    reps_c = max(2, reps // 4)
+    out["chunked_attn_ms"] = _time_calls(torch, stream, chunked, reps_c)
+    out["merge_ms"] = _time_calls(torch, stream, merge, reps)
     return out
 
 
-def cache_rows_report(extra, fcase, case, peaks):
+def next_rows_report(extra, fcase, case, peaks):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     n = fcase.n
     o_elems = case.B * case.H * case.N * case.d
@@ -324,6 +349,12 @@ def cache_rows_report(extra, fcase, case, peaks):
                                  f"bf16 vs 8-bit attention output, {case.B * case.H} segments"),
         "graph_step": {"cached_ms": extra["graph_cached_step_ms"], "computed_ms": extra["graph_computed_step_ms"],
                        "what": "fbcache_step + IF node over one bf16 attention call; body skipped vs run"},
+        "attn_merge": hbm_row(extra["merge_ms"], CHUNKS * (o_elems * 2 + o_elems // case.d * 4)
+                              + o_elems * 2 + o_elems // case.d * 4,
+                              f"read {CHUNKS} chunk outputs (bf16) and log-sum-exps, write output and log-sum-exp"),
+        "chunked_attn": {"ms": extra["chunked_attn_ms"], "chunks": CHUNKS,
+                         "tflops": case.flops / (extra["chunked_attn_ms"] * 1e-3) / 1e12,
+                         "what": f"{CHUNKS} x dit_attn_fwd_ex over key chunks with log-sum-exp (merge excluded)"},
     }
 
 
@@ -465,7 +496,7 @@ def run_ours(args):
     prepass_ms = ep[0].elapsed_time(ep[1]) / K
 
     # ---- the step caches and the output comparison (outside the timed step)
-    extra = measure_cache_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk, dv, case, K)
+    extra = measure_next_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk, dv, case, K)
 
     # ---- max over ranks
     keys = sorted(extra)
@@ -503,7 +534,7 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
-        "cache_rows": cache_rows_report(extra, fcase, case, peaks),
+        "next_rows": next_rows_report(extra, fcase, case, peaks),
     }
     roof_bf16 = {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                  "frac": attn_tflops / peak,

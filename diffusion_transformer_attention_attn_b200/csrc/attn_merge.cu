@@ -10,10 +10,10 @@
 // which is the attention over the union of the keys.
 //
 // HBM-bound: each thread owns one 16-byte slice (8 channels) of one query
-// row, reads the row's L_c (shared by the slices of the row, served from L1),
-// forms the weights with the largest L_c subtracted first, then streams the
-// matching slice of every O_c and writes the bf16 result.  The first slice of
-// a row also writes L.
+// row.  It issues the loads of the row's L_c (shared by the slices of the
+// row, served from L1) and of the matching slice of every O_c together, forms
+// the weights with the largest L_c subtracted first, and writes the bf16
+// result.  The first slice of a row also writes L.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -33,9 +33,12 @@ struct MergeParts {
     const float* lse[kMaxMergeParts];
 };
 
+// NP: the number of parts (a template argument, so that every part's loads
+// are issued before any of them is used).
+template <int NP>
 __global__ void __launch_bounds__(kMergeThreads)
-    attn_merge_kernel(MergeParts parts, int n_parts, int64_t rows, int H, int N, int d, int64_t sb, int64_t sh,
-                      int64_t sn, __nv_bfloat16* __restrict__ o, float* __restrict__ lse_out) {
+    attn_merge_kernel(MergeParts parts, int64_t rows, int H, int N, int d, int64_t sb, int64_t sh, int64_t sn,
+                      __nv_bfloat16* __restrict__ o, float* __restrict__ lse_out) {
     const int slices = d / 8;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (t >= rows * slices) return;
@@ -46,25 +49,26 @@ __global__ void __launch_bounds__(kMergeThreads)
     const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
     const int64_t off = b * sb + h * sh + static_cast<int64_t>(n) * sn + sl * 8;
 
-    float L[kMaxMergeParts];
-    float lmax = -INFINITY;
+    float L[NP];
+    uint4 v[NP];
 #pragma unroll
-    for (int c = 0; c < kMaxMergeParts; ++c) {
-        L[c] = c < n_parts ? __ldg(parts.lse[c] + r) : -INFINITY;
-        lmax = fmaxf(lmax, L[c]);
+    for (int c = 0; c < NP; ++c) {
+        L[c] = __ldg(parts.lse[c] + r);
+        v[c] = __ldcs(reinterpret_cast<const uint4*>(parts.o[c] + off));
     }
+    float lmax = L[0];
+#pragma unroll
+    for (int c = 1; c < NP; ++c) lmax = fmaxf(lmax, L[c]);
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     float wsum = 0.f;
     if (lmax > -INFINITY) {
 #pragma unroll
-        for (int c = 0; c < kMaxMergeParts; ++c) {
-            if (c >= n_parts) break;
+        for (int c = 0; c < NP; ++c) {
             const float w = expf(L[c] - lmax);
             wsum += w;
-            const uint4 v = __ldcs(reinterpret_cast<const uint4*>(parts.o[c] + off));
-            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t u[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
@@ -79,8 +83,28 @@ __global__ void __launch_bounds__(kMergeThreads)
         const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * i] * inv, acc[2 * i + 1] * inv);
         pk[i] = *reinterpret_cast<const uint32_t*>(&p);
     }
-    *reinterpret_cast<uint4*>(o + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    __stcs(reinterpret_cast<uint4*>(o + off), make_uint4(pk[0], pk[1], pk[2], pk[3]));
     if (lse_out != nullptr && sl == 0) lse_out[r] = wsum > 0.f ? lmax + logf(wsum) : -INFINITY;
+}
+
+template <int NP>
+cudaError_t launch_np(const MergeParts& p, int64_t rows, int H, int N, int d, int64_t sb, int64_t sh, int64_t sn,
+                      void* o, float* lse, cudaStream_t stream) {
+    const int64_t threads = rows * (d / 8);
+    const int64_t blocks = (threads + kMergeThreads - 1) / kMergeThreads;
+    if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    attn_merge_kernel<NP><<<static_cast<unsigned>(blocks), kMergeThreads, 0, stream>>>(
+        p, rows, H, N, d, sb, sh, sn, static_cast<__nv_bfloat16*>(o), lse);
+    return cudaGetLastError();
+}
+
+template <int NP>
+cudaError_t dispatch(int n_parts, const MergeParts& p, int64_t rows, int H, int N, int d, int64_t sb, int64_t sh,
+                     int64_t sn, void* o, float* lse, cudaStream_t stream) {
+    if (n_parts == NP) return launch_np<NP>(p, rows, H, N, d, sb, sh, sn, o, lse, stream);
+    if constexpr (NP < kMaxMergeParts)
+        return dispatch<NP + 1>(n_parts, p, rows, H, N, d, sb, sh, sn, o, lse, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -94,12 +118,7 @@ cudaError_t launch_attn_merge(const void* const* o_parts, const float* const* ls
         p.lse[c] = c < n_parts ? lse_parts[c] : nullptr;
     }
     const int64_t rows = static_cast<int64_t>(B) * H * N;
-    const int64_t threads = rows * (d / 8);
-    const int64_t blocks = (threads + kMergeThreads - 1) / kMergeThreads;
-    if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    attn_merge_kernel<<<static_cast<unsigned>(blocks), kMergeThreads, 0, stream>>>(
-        p, n_parts, rows, H, N, d, sb, sh, sn, static_cast<__nv_bfloat16*>(o), lse);
-    return cudaGetLastError();
+    return dispatch<1>(n_parts, p, rows, H, N, d, sb, sh, sn, o, lse, stream);
 }
 
 }  // namespace ditk
