@@ -13,6 +13,12 @@
 #include "dit_attn.h"
 #include "internal.h"
 
+#ifdef DIT_ATTN_KS
+#define ATTN_BF16_LAUNCH launch_attn_bf16_ks
+#else
+#define ATTN_BF16_LAUNCH launch_attn_bf16
+#endif
+
 namespace ditk {
 
 // Device-side error word (one per device that loads the library); kernels
@@ -231,7 +237,7 @@ dit_status dit_attn_fwd_ex(const void* q, const void* k, const void* v, void* o,
     if ((st = encode_bf16_map(&tv, v, B, H, Nkv, d, kb, kh, kn)) != DIT_OK) return st;
     const float s = scale > 0.f ? scale : default_scale(d);
     const float scale_log2 = static_cast<float>(static_cast<double>(s) * 1.4426950408889634);
-    cudaError_t e = launch_attn_bf16(tq, tk, tv, o, qb, qh, qn, B, H, Nq, Nkv, d, scale_log2, lse, ds->err_word,
+    cudaError_t e = ATTN_BF16_LAUNCH(tq, tk, tv, o, qb, qh, qn, B, H, Nq, Nkv, d, scale_log2, lse, ds->err_word,
                                      static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
@@ -279,7 +285,7 @@ dit_status dit_attn_fwd(const void* q, const void* k, const void* v, void* o, in
     if ((st = encode_bf16_map(&tv, v, B, H, N, d, sb, sh, sn)) != DIT_OK) return st;
     const float s = scale > 0.f ? scale : default_scale(d);
     const float scale_log2 = static_cast<float>(static_cast<double>(s) * 1.4426950408889634);
-    cudaError_t e = launch_attn_bf16(tq, tk, tv, o, sb, sh, sn, B, H, N, N, d, scale_log2, nullptr, ds->err_word,
+    cudaError_t e = ATTN_BF16_LAUNCH(tq, tk, tv, o, sb, sh, sn, B, H, N, N, d, scale_log2, nullptr, ds->err_word,
                                      static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }

@@ -236,13 +236,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = mbar_wait(bars.q_full, 0, abort_flag, err) && mbar_wait(&bars.k_full[0], 0, abort_flag, err);
         if (ok) {
             tc_fence_after();
-            if (lane == 0) {
-                issue_s(tS0, dQ0, dK0);
-                mma_commit(&bars.s_full[0]);
-                issue_s(tS1, dQ1, dK0);
-                mma_commit(&bars.s_full[1]);
-                mma_commit(&bars.k_empty[0]);
-            }
+            issue_s(tS0, dQ0, dK0);
+            mma_commit(&bars.s_full[0]);
+            issue_s(tS1, dQ1, dK0);
+            mma_commit(&bars.s_full[1]);
+            mma_commit(&bars.k_empty[0]);
             __syncwarp();
             for (int j = 0; j < nkv && ok; ++j) {
                 const int vs = j % C::kStages;
@@ -260,47 +258,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = ok && mbar_wait(&bars.p_full[2 * t + hf], j & 1, abort_flag, err);
                         if (!ok) return;
                         tc_fence_after();
-                        if (lane == 0) {
 #pragma unroll
-                            for (int kk = hf * (8 / kParts); kk < (hf + 1) * (8 / kParts); ++kk)
-                                mma_ts<0>(tO, tP + kk * 8, sdesc_add(dV, v_off(kk)), C::kIdescPV, (j > 0 || kk > 0));
-                        }
+                        for (int kk = hf * (8 / kParts); kk < (hf + 1) * (8 / kParts); ++kk)
+                            mma_ts<0>(tO, tP + kk * 8, sdesc_add(dV, v_off(kk)), C::kIdescPV, (j > 0 || kk > 0));
                         __syncwarp();
                     }
                 };
                 issue_pv(0, tO0, tS0);
                 if (!ok) break;
-                if (lane == 0) mma_commit(&bars.o_ready[0]);
+                mma_commit(&bars.o_ready[0]);
                 __syncwarp();
                 if (more) {
                     ok = mbar_wait(&bars.k_full[ks], ((j + 1) / C::kStages) & 1, abort_flag, err);
                     if (!ok) break;
                     tc_fence_after();
-                    if (lane == 0) {
-                        issue_s(tS0, dQ0, dK);
-                        mma_commit(&bars.s_full[0]);
-                    }
+                    issue_s(tS0, dQ0, dK);
+                    mma_commit(&bars.s_full[0]);
                     __syncwarp();
                 }
                 issue_pv(1, tO1, tS1);
                 if (!ok) break;
-                if (lane == 0) {
-                    mma_commit(&bars.o_ready[1]);
-                    mma_commit(&bars.v_empty[vs]);
-                    if (more) {
-                        issue_s(tS1, dQ1, dK);
-                        mma_commit(&bars.s_full[1]);
-                        mma_commit(&bars.k_empty[ks]);
-                    }
+                mma_commit(&bars.o_ready[1]);
+                mma_commit(&bars.v_empty[vs]);
+                if (more) {
+                    issue_s(tS1, dQ1, dK);
+                    mma_commit(&bars.s_full[1]);
+                    mma_commit(&bars.k_empty[ks]);
                 }
                 __syncwarp();
             }
         }
         // Every MMA issued above has completed once mma_done flips.
-        if (lane == 0) {
-            mma_commit(bars.mma_done);
-            mbar_wait_drain(bars.mma_done, 0);
-        }
+        mma_commit(bars.mma_done);
+        if (lane == 0) mbar_wait_drain(bars.mma_done, 0);
         __syncwarp();
       }
     } else {

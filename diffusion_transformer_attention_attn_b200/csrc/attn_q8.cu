@@ -220,13 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = mbar_wait(bars.q_full, 0, abort_flag, err) && mbar_wait(&bars.k_full[0], 0, abort_flag, err);
             if (ok) {
                 tc_fence_after();
-                if (lane == 0) {
-                    issue_s(tS0, dQ0, dK0);
-                    mma_commit(&bars.s_full[0]);
-                    issue_s(tS1, dQ1, dK0);
-                    mma_commit(&bars.s_full[1]);
-                    mma_commit(&bars.k_empty[0]);
-                }
+                issue_s(tS0, dQ0, dK0);
+                mma_commit(&bars.s_full[0]);
+                issue_s(tS1, dQ1, dK0);
+                mma_commit(&bars.s_full[1]);
+                mma_commit(&bars.k_empty[0]);
                 __syncwarp();
                 for (int j = 0; j < nkv && ok; ++j) {
                     const int vs = j % C::kStages;
@@ -238,41 +236,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                          mbar_wait(&bars.p_full[0], j & 1, abort_flag, err);
                     if (!ok) break;
                     tc_fence_after();
-                    if (lane == 0) {
-                        issue_pv(tO0, tS0, dV, j > 0);
-                        mma_commit(&bars.o_ready[0]);
-                    }
+                    issue_pv(tO0, tS0, dV, j > 0);
+                    mma_commit(&bars.o_ready[0]);
                     __syncwarp();
                     if (more) {
                         ok = mbar_wait(&bars.k_full[ks], ((j + 1) / C::kStages) & 1, abort_flag, err);
                         if (!ok) break;
                         tc_fence_after();
-                        if (lane == 0) {
-                            issue_s(tS0, dQ0, dK);
-                            mma_commit(&bars.s_full[0]);
-                        }
+                        issue_s(tS0, dQ0, dK);
+                        mma_commit(&bars.s_full[0]);
                         __syncwarp();
                     }
                     ok = mbar_wait(&bars.p_full[1], j & 1, abort_flag, err);
                     if (!ok) break;
                     tc_fence_after();
-                    if (lane == 0) {
-                        issue_pv(tO1, tS1, dV, j > 0);
-                        mma_commit(&bars.o_ready[1]);
-                        mma_commit(&bars.v_empty[vs]);
-                        if (more) {
-                            issue_s(tS1, dQ1, dK);
-                            mma_commit(&bars.s_full[1]);
-                            mma_commit(&bars.k_empty[ks]);
-                        }
+                    issue_pv(tO1, tS1, dV, j > 0);
+                    mma_commit(&bars.o_ready[1]);
+                    mma_commit(&bars.v_empty[vs]);
+                    if (more) {
+                        issue_s(tS1, dQ1, dK);
+                        mma_commit(&bars.s_full[1]);
+                        mma_commit(&bars.k_empty[ks]);
                     }
                     __syncwarp();
                 }
             }
-            if (lane == 0) {
-                mma_commit(bars.mma_done);
-                mbar_wait_drain(bars.mma_done, 0);
-            }
+            mma_commit(bars.mma_done);
+            if (lane == 0) mbar_wait_drain(bars.mma_done, 0);
             __syncwarp();
         }
     } else {

@@ -18,6 +18,12 @@ cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const
                              int64_t sb, int64_t sh, int64_t sn, int B, int H, int Nq, int Nkv, int d,
                              float scale_log2, float* lse, int* err, cudaStream_t stream);
 
+// The same attention with one 128-row query tile per CTA and the keys of each
+// tile split between two softmax warpgroups (attn_bf16_ks.cu).
+cudaError_t launch_attn_bf16_ks(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                                int64_t sb, int64_t sh, int64_t sn, int B, int H, int Nq, int Nkv, int d,
+                                float scale_log2, float* lse, int* err, cudaStream_t stream);
+
 // Merge of per-key-chunk outputs (see dit_attn_merge in dit_attn.h).
 constexpr int kMaxMergeParts = 16;
 cudaError_t launch_attn_merge(const void* const* o_parts, const float* const* lse_parts, int n_parts, int B, int H,

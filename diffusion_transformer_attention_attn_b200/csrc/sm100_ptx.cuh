@@ -198,23 +198,33 @@ __device__ __forceinline__ SDesc sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes,
 }
 __device__ __forceinline__ SDesc sdesc_add(SDesc d, uint32_t bytes) { return SDesc{d.lo + (bytes >> 4), d.hi}; }
 
+// MMA issue is warp-collective: every lane of the (converged) issuing warp
+// executes these with warp-uniform operands, and elect.sync picks the one lane
+// that issues the instruction.  The same lane (the lowest, all lanes being
+// active) issues every MMA and every commit, so a commit covers all MMAs the
+// warp issued before it.  Issuing this way keeps the operands on the uniform
+// datapath; guarding a single-thread issue with `lane == 0` made each MMA issue
+// take 80-110 cycles next to busy softmax warps instead of about 40-60.
+//
 // D[tmem] (+)= A[smem] · B[smem] (kind::f16 / kind::i8), split descriptors.
 template <int KIND>  // 0: f16 (bf16 in, fp32 acc), 1: i8 (s8 in, s32 acc)
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, SDesc a, SDesc b, uint32_t idesc, uint32_t accumulate) {
     if (KIND == 0)
         asm volatile(
-            "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+            "{\n\t.reg .pred p, e;\n\t.reg .b64 da, db;\n\t"
+            "elect.sync _|e, 0xffffffff;\n\t"
             "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
             "setp.ne.b32 p, %6, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+            "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
             "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
             : "memory");
     else
         asm volatile(
-            "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+            "{\n\t.reg .pred p, e;\n\t.reg .b64 da, db;\n\t"
+            "elect.sync _|e, 0xffffffff;\n\t"
             "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
             "setp.ne.b32 p, %6, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::i8 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+            "@e tcgen05.mma.cta_group::1.kind::i8 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
             "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
             : "memory");
 }
@@ -224,48 +234,30 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, SDesc b
                                        uint32_t accumulate) {
     if (KIND == 0)
         asm volatile(
-            "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+            "{\n\t.reg .pred p, e;\n\t.reg .b64 db;\n\t"
+            "elect.sync _|e, 0xffffffff;\n\t"
             "mov.b64 db, {%2, %3};\n\t"
             "setp.ne.b32 p, %5, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+            "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
             "r"(a_tmem), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
             : "memory");
     else
         asm volatile(
-            "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+            "{\n\t.reg .pred p, e;\n\t.reg .b64 db;\n\t"
+            "elect.sync _|e, 0xffffffff;\n\t"
             "mov.b64 db, {%2, %3};\n\t"
             "setp.ne.b32 p, %5, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+            "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
             "r"(a_tmem), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
             : "memory");
 }
-
-// D[tmem] (+)= A[smem] · B[smem], bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// D[tmem] (+)= A[tmem] · B[smem], bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// Arrive (once) on `bar` when every tcgen05 operation this thread issued so
-// far has completed.
+// Arrive (once) on `bar` when every tcgen05 operation the issuing lane started
+// so far has completed (warp-collective, like the MMAs).
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
 }
 
 // ---------------------------------------------------------------- registers
