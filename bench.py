@@ -45,11 +45,11 @@ METRIC = "attention TFLOPS (4·B·H·N²·d/s) and % of B200 tensor peak at N=11
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
-# DRAM bytes (read + write) of one launch, from the ncu capture summarised in
-# profiles/attn_fwd_bf16_video_mid_n45760.md (N=45760, 24 heads), scaled by N:
+# DRAM bytes (read + write) of one launch of the bf16 attention kernel, from an
+# ncu capture on the 45760-token, 24-head video workload, scaled by N:
 # each head's K/V stays L2-resident while its CTAs run, so traffic grows with N.
 # Set to None whenever the kernel changes until it is captured again.
-BF16_ATTN_DRAM_BYTES_AT = (1.134775e9, 45760)
+BF16_ATTN_DRAM_BYTES_AT = (1.126394e9, 45760)
 SPEC_HBM_GBS = 8000.0
 
 
@@ -496,7 +496,8 @@ def run_ours(args):
     prepass_ms = ep[0].elapsed_time(ep[1]) / K
 
     # ---- the step caches and the output comparison (outside the timed step)
-    extra = measure_next_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk, dv, case, K)
+    extra = {} if args.no_next_rows else measure_next_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk,
+                                                                 dv, case, K)
 
     # ---- max over ranks
     keys = sorted(extra)
@@ -534,7 +535,7 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
-        "next_rows": next_rows_report(extra, fcase, case, peaks),
+        "next_rows": None if args.no_next_rows else next_rows_report(extra, fcase, case, peaks),
     }
     roof_bf16 = {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                  "frac": attn_tflops / peak,
@@ -585,6 +586,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="video_long",
                     help="video_long is the benchmark; the others serve profiling captures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the step-cache, comparison, merge and chunked-attention timings")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
