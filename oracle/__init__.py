@@ -278,3 +278,23 @@ def merge_partials(outs, lses):
     den = w.sum(axis=0)
     out = (w[..., None] * O).sum(axis=0) / den[..., None]
     return out, top + np.log(den)
+
+
+def fbc_sums(cur, prev):
+    """(sum|cur - prev|, sum|prev|) in fp64: the two sums behind fbc_rel_l1.
+
+    A residual split across devices reduces to rel with one all-reduce of
+    these two numbers (ParaAttention page, "First Block Cache", with the
+    residual sharded as the sequence is in "Context Parallelism")."""
+    c = _widen(np.ascontiguousarray(cur).reshape(-1))
+    p = _widen(np.ascontiguousarray(prev).reshape(-1))
+    return float(np.abs(c - p).sum()), float(np.abs(p).sum())
+
+
+def rel_from_sums(num: float, den: float, threshold: float):
+    """(rel, skip) from the two sums, with fbc_rel_l1's conventions."""
+    if den > 0:
+        rel = num / den
+    else:
+        rel = float("inf") if num > 0 else 0.0
+    return rel, int(rel < float(np.float32(threshold)))

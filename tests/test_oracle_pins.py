@@ -364,3 +364,20 @@ def test_fp8_value_rounding_floor():
     kd = kc * ks[:, :, tok // 64, None].astype(np.float64)
     rel_qk = np.abs(oracle.attention(qd, kd, f(v), rows=rows) - ref).sum() / np.abs(ref).sum()
     assert 0.005 < rel_qk < 0.02
+
+
+def test_fbc_sums_of_shards_add_up_and_give_rel():
+    rng = np.random.default_rng(11)
+    prev = rng.standard_normal(10007).astype(np.float32)
+    cur = (prev + 0.05 * rng.standard_normal(prev.size)).astype(np.float32)
+    num, den = oracle.fbc_sums(cur, prev)
+    parts = [oracle.fbc_sums(cur[a:b], prev[a:b]) for a, b in ((0, 3000), (3000, 3001), (3001, 10007))]
+    assert abs(sum(x for x, _ in parts) - num) <= 1e-9 * num
+    assert abs(sum(y for _, y in parts) - den) <= 1e-9 * den
+    rel, skip = oracle.rel_from_sums(num, den, 0.08)
+    rel_ref, skip_ref = oracle.fbc_rel_l1(cur, prev, 0.08)
+    assert abs(rel - rel_ref) <= 1e-12 * rel_ref and skip == skip_ref
+    # the hand case of the First Block Cache reading: 1.5 / 10
+    assert oracle.fbc_sums(np.float32([1.5, -2, 2, -4]), np.float32([1, -2, 3, -4])) == (1.5, 10.0)
+    assert oracle.rel_from_sums(0.0, 0.0, 0.1) == (0.0, 1)
+    assert oracle.rel_from_sums(1.0, 0.0, 0.1) == (float("inf"), 0)
