@@ -330,6 +330,49 @@ def measure_next_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk, dv,
     reps_c = max(2, reps // 4)
     out["chunked_attn_ms"] = _time_calls(torch, stream, chunked, reps_c)
     out["merge_ms"] = _time_calls(torch, stream, merge, reps)
+    del parts, mo, ml
+
+    # fbc_rel_l1 at the image workload's residual size (4608x3072 bf16, 56.6 MB
+    # per pair, below L2): a CUDA graph of 50 launches rotating over 5 pairs
+    # (283 MB, more than twice L2) for GB/s, and single launches for latency.
+    fc = inputs.FBC_IMAGE
+    pairs = []
+    for r in range(5):
+        c, p = inputs.fbc_inputs(inputs.FbcCase(f"fbc_rot{r}", fc.rows, fc.cols, "bf16", fc.drift_std, fc.threshold,
+                                                seed=100 + r))
+        pairs.append(tuple(torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in (c, p)))
+    fws = dit.fbc_workspace(fc.n, dev)
+    rel = torch.empty(1, dtype=torch.float64, device=dev)
+    skip = torch.empty(1, dtype=torch.int32, device=dev)
+    for c, p in pairs:
+        dit.fbc_rel_l1(c, p, fc.threshold, out_rel=rel, out_skip=skip, workspace=fws)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    gs = torch.cuda.Stream(dev)
+    with torch.cuda.graph(g, stream=gs):
+        for i in range(50):
+            c, p = pairs[i % 5]
+            dit.fbc_rel_l1(c, p, fc.threshold, out_rel=rel, out_skip=skip, workspace=fws)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    ge = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ge[0].record(stream)
+    for _ in range(4):
+        g.replay()
+    ge[1].record(stream)
+    ge[1].synchronize()
+    out["fbc_image_graph_ms_per_launch"] = ge[0].elapsed_time(ge[1]) / 200
+    lat = []
+    for i in range(20):
+        c, p = pairs[i % 5]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        dit.fbc_rel_l1(c, p, fc.threshold, out_rel=rel, out_skip=skip, workspace=fws)
+        e[1].record(stream)
+        e[1].synchronize()
+        lat.append(e[0].elapsed_time(e[1]))
+    out["fbc_image_single_launch_ms"] = statistics.median(lat)
+    del g, pairs
     return out
 
 
@@ -352,6 +395,10 @@ def next_rows_report(extra, fcase, case, peaks):
         "attn_merge": hbm_row(extra["merge_ms"], CHUNKS * (o_elems * 2 + o_elems // case.d * 4)
                               + o_elems * 2 + o_elems // case.d * 4,
                               f"read {CHUNKS} chunk outputs (bf16) and log-sum-exps, write output and log-sum-exp"),
+        "fbc_image": dict(hbm_row(extra["fbc_image_graph_ms_per_launch"], 2 * inputs.FBC_IMAGE.n * 2,
+                                  "fbc_rel_l1 on 4608x3072 bf16: CUDA graph of 50 launches over 5 residual pairs "
+                                  "(283 MB, > 2x L2)"),
+                          single_launch_latency_ms=extra["fbc_image_single_launch_ms"]),
         "chunked_attn": {"ms": extra["chunked_attn_ms"], "chunks": CHUNKS,
                          "tflops": case.flops / (extra["chunked_attn_ms"] * 1e-3) / 1e12,
                          "what": f"{CHUNKS} x dit_attn_fwd_ex over key chunks with log-sum-exp (merge excluded)"},

@@ -58,6 +58,8 @@ SIGNATURES = {
     "fbc_rel_l1_workspace_bytes": (_sz, [_i64]),
     "fbc_rel_l1": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p, _sz, _p]),
     "fbc_rel_l1_noalloc": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p]),
+    "fbc_rel_l1_sums": (_i, [_p, _p, _i64, _i, _p, _p, _sz, _p]),
+    "fbc_rel_l1_finish": (_i, [_p, _f, _p, _p, _p]),
     "dit_compare_workspace_bytes": (_sz, [_i64, _i64, _i]),
     "dit_compare_stats": (_i, [_p, _p, _i64, _i64, _i, _p, _p, _sz, _p]),
     "dit_get_device_status": (_i, [_p]),
@@ -340,6 +342,40 @@ def fbc_rel_l1(r_cur, r_prev, threshold: float, out_rel=None, out_skip=None, wor
     st = lib.fbc_rel_l1(r_cur.data_ptr(), r_prev.data_ptr(), n, dt, float(threshold), out_rel.data_ptr(),
                         out_skip.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
     _check(st, "fbc_rel_l1")
+    return out_rel, out_skip
+
+
+def fbc_rel_l1_sums(r_cur, r_prev, out_sums=None, workspace=None, stream=None):
+    """Σ|r_cur − r_prev| and Σ|r_prev| over these tensors (device float64[2])."""
+    import torch
+    lib = load_library()
+    if r_cur.shape != r_prev.shape or r_cur.dtype != r_prev.dtype:
+        raise ValueError("r_cur and r_prev must match in shape and dtype")
+    if not (r_cur.is_contiguous() and r_prev.is_contiguous()):
+        raise ValueError("r_cur and r_prev must be contiguous")
+    dt = _dtype_code(r_cur, "fbc_rel_l1_sums")
+    n = r_cur.numel()
+    if out_sums is None:
+        out_sums = torch.empty(2, dtype=torch.float64, device=r_cur.device)
+    if workspace is None:
+        workspace = fbc_workspace(n, r_cur.device)
+    st = lib.fbc_rel_l1_sums(r_cur.data_ptr(), r_prev.data_ptr(), n, dt, out_sums.data_ptr(), workspace.data_ptr(),
+                             workspace.numel(), _stream_ptr(stream))
+    _check(st, "fbc_rel_l1_sums")
+    return out_sums
+
+
+def fbc_rel_l1_finish(sums, threshold: float, out_rel=None, out_skip=None, stream=None):
+    """(rel, skip) device tensors from a float64[2] sums tensor."""
+    import torch
+    lib = load_library()
+    if out_rel is None:
+        out_rel = torch.empty(1, dtype=torch.float64, device=sums.device)
+    if out_skip is None:
+        out_skip = torch.empty(1, dtype=torch.int32, device=sums.device)
+    st = lib.fbc_rel_l1_finish(sums.data_ptr(), float(threshold), out_rel.data_ptr(), out_skip.data_ptr(),
+                               _stream_ptr(stream))
+    _check(st, "fbc_rel_l1_finish")
     return out_rel, out_skip
 
 

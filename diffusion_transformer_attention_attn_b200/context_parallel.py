@@ -1,10 +1,10 @@
 """Context parallelism for the attention call: one process per GPU, the token
 sequence split evenly across the ranks of a ``torch.distributed`` group.
 
-Two schemes, both from "ParaAttention" (diffusers docs), section "Context
-Parallelism", and the TMAP image-to-video blog, section on sequence
+Two attention schemes, both from "ParaAttention" (diffusers docs), section
+"Context Parallelism", and the TMAP image-to-video blog, section on sequence
 parallelism (Ulysses, with its all-to-all overlapped with the surrounding
-work):
+work), and the cache decision over a sharded residual:
 
 * ``ulysses_attention`` — each rank holds all heads of its N/P tokens.  One
   all-to-all regroups Q, K and V so that each rank holds H/P heads of all N
@@ -14,10 +14,15 @@ work):
   around the ring; every step attends the local queries to the chunk in hand
   (``dit_attn_fwd_ex`` with log-sum-exp), while the next chunk is already in
   flight, and the per-chunk results are merged (``dit_attn_merge``).
+* ``sharded_fbc_rel_l1`` — the first-block-cache difference of a residual
+  sharded like the sequence: each rank reduces its slice to two sums
+  (``fbc_rel_l1_sums``), one all-reduce adds them, and ``fbc_rel_l1_finish``
+  forms rel and the decision on every rank.
 
-The collectives are torch.distributed calls (NCCL between GPUs); the attention
-and the merge are the library's kernels.  ``attn_fn`` / ``attn_lse_fn`` /
-``merge_fn`` may be replaced, e.g. to run the data movement on CPU ranks.
+The collectives are torch.distributed calls (NCCL between GPUs); the attention,
+the merge and the reductions are the library's kernels.  ``attn_fn``,
+``attn_lse_fn``, ``merge_fn``, ``sums_fn`` and ``finish_fn`` may be replaced,
+e.g. to run the data movement on CPU ranks.
 """
 from __future__ import annotations
 
@@ -129,3 +134,24 @@ def ring_attention(q, k, v, group=None, attn_lse_fn=None, merge_fn=None):
     if len(outs) == 1:
         return outs[0], lses[0]
     return merge(outs, lses)
+
+
+def _default_sums(cur, prev):
+    from . import fbc_rel_l1_sums
+    return fbc_rel_l1_sums(cur, prev)
+
+
+def _default_finish(sums, threshold):
+    from . import fbc_rel_l1_finish
+    return fbc_rel_l1_finish(sums, threshold)
+
+
+def sharded_fbc_rel_l1(r_cur, r_prev, threshold: float, group=None, sums_fn=None, finish_fn=None):
+    """(rel, skip) of a residual whose elements are split across the ranks of
+    ``group``; every rank gets the same result."""
+    import torch.distributed as dist
+    sums = (sums_fn or _default_sums)(r_cur, r_prev)
+    world, _ = _group_info(group)
+    if world > 1:
+        dist.all_reduce(sums, op=dist.ReduceOp.SUM, group=group)
+    return (finish_fn or _default_finish)(sums, threshold)

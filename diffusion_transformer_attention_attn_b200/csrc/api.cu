@@ -375,6 +375,32 @@ dit_status fbc_rel_l1(const void* r_cur, const void* r_prev, int64_t n, int dtyp
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
+dit_status fbc_rel_l1_sums(const void* r_cur, const void* r_prev, int64_t n, int dtype, double* out_sums,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    if (!r_cur || !r_prev || !out_sums || n < 1) return DIT_ERR_INVALID_ARG;
+    if (dtype != DIT_DTYPE_F32 && dtype != DIT_DTYPE_BF16) return DIT_ERR_INVALID_ARG;
+    if (!aligned16(r_cur) || !aligned16(r_prev) || (reinterpret_cast<uintptr_t>(out_sums) & 7u) != 0)
+        return DIT_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < fbc_workspace_bytes(n)) return DIT_ERR_WORKSPACE;
+    dit_status st;
+    if (!device_state(&st)) return st;
+    cudaError_t e = launch_fbc_sums(r_cur, r_prev, n, dtype, out_sums, workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+dit_status fbc_rel_l1_finish(const double* sums, float threshold, double* out_rel, int32_t* out_skip,
+                             void* stream) {
+    if (!sums || !out_rel || !out_skip) return DIT_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(sums) & 7u) != 0 || (reinterpret_cast<uintptr_t>(out_rel) & 7u) != 0 ||
+        (reinterpret_cast<uintptr_t>(out_skip) & 3u) != 0)
+        return DIT_ERR_INVALID_ARG;
+    if (!(threshold == threshold)) return DIT_ERR_INVALID_ARG;
+    dit_status st;
+    if (!device_state(&st)) return st;
+    cudaError_t e = launch_fbc_finish(sums, threshold, out_rel, out_skip, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
 dit_status dit_get_device_status(void* stream) {
     dit_status st;
     DeviceState* ds = device_state(&st);

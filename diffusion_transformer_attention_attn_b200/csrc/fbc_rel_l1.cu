@@ -31,6 +31,25 @@ struct EpiThreshold {
     }
 };
 
+// The two sums themselves (for a residual sharded across devices).
+struct EpiSums {
+    double* out;
+    __device__ bool evaluate() const { return true; }
+    __device__ void finish(double num, double den, bool) const {
+        out[0] = num;
+        out[1] = den;
+    }
+};
+
+__global__ void fbc_finish_kernel(const double* __restrict__ sums, float threshold, double* __restrict__ out_rel,
+                                  int32_t* __restrict__ out_skip) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+        const double rel = rl1_ratio(sums[0], sums[1]);
+        *out_rel = rel;
+        *out_skip = (rel < static_cast<double>(threshold)) ? 1 : 0;
+    }
+}
+
 }  // namespace
 
 size_t fbc_workspace_bytes(int64_t /*n*/) {
@@ -40,6 +59,17 @@ size_t fbc_workspace_bytes(int64_t /*n*/) {
 cudaError_t launch_fbc_rel_l1(const void* cur, const void* prev, int64_t n, int dtype, float threshold,
                               double* out_rel, int32_t* out_skip, void* workspace, cudaStream_t stream) {
     return launch_rel_l1<false>(cur, prev, n, dtype, EpiThreshold{threshold, out_rel, out_skip}, workspace, stream);
+}
+
+cudaError_t launch_fbc_sums(const void* cur, const void* prev, int64_t n, int dtype, double* out_sums,
+                            void* workspace, cudaStream_t stream) {
+    return launch_rel_l1<false>(cur, prev, n, dtype, EpiSums{out_sums}, workspace, stream);
+}
+
+cudaError_t launch_fbc_finish(const double* sums, float threshold, double* out_rel, int32_t* out_skip,
+                              cudaStream_t stream) {
+    fbc_finish_kernel<<<1, 32, 0, stream>>>(sums, threshold, out_rel, out_skip);
+    return cudaGetLastError();
 }
 
 }  // namespace ditk

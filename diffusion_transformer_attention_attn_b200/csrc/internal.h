@@ -63,5 +63,9 @@ dit_status check_device();
 size_t fbc_workspace_bytes(int64_t n);
 cudaError_t launch_fbc_rel_l1(const void* cur, const void* prev, int64_t n, int dtype, float threshold,
                               double* out_rel, int32_t* out_skip, void* workspace, cudaStream_t stream);
+cudaError_t launch_fbc_sums(const void* cur, const void* prev, int64_t n, int dtype, double* out_sums,
+                            void* workspace, cudaStream_t stream);
+cudaError_t launch_fbc_finish(const double* sums, float threshold, double* out_rel, int32_t* out_skip,
+                              cudaStream_t stream);
 
 }  // namespace ditk

@@ -12,8 +12,9 @@
 // elements and folds into fp64; blocks reduce in fp64 with warp shuffles.
 // Each block writes its partial pair to the workspace; the last block to take
 // a ticket adds the partials in block order, runs the epilogue and re-zeroes
-// the ticket.  The grid size depends on n only, so the summation order, and
-// the result, are the same on every run.
+// the ticket.  The grid (at most one wave of resident blocks) depends on n
+// and the GPU's SM count only, so the summation order, and the result, are
+// the same on every run on a given device.
 //
 // With kCopy the kernel also stores cur into prev in the same pass (each
 // element is read before the same thread overwrites it), the update that the
@@ -167,11 +168,31 @@ __global__ void __launch_bounds__(kFbcThreads)
     }
 }
 
+// Blocks of kFbcThreads that fit on the current GPU at once (4 per SM on
+// sm_100: 2048 threads), queried once per device.
+inline int rel_l1_resident_blocks() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kFbcMaxBlocks;
+    if (cached[dev] == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+            return kFbcMaxBlocks;
+        cached[dev] = sms * (2048 / kFbcThreads);
+    }
+    return cached[dev];
+}
+
+// One wave of resident blocks at most (more only adds a partial second wave),
+// never more than the workspace holds.  The grid depends on n and the GPU's
+// SM count only, so a given device always sums in the same order.
 inline int rel_l1_blocks(int64_t nvec) {
     const int64_t per = static_cast<int64_t>(kFbcThreads) * kFbcUnroll;
     int64_t nb = (nvec + per - 1) / per;
+    int64_t cap = rel_l1_resident_blocks();
+    if (cap > kFbcMaxBlocks) cap = kFbcMaxBlocks;
     if (nb < 1) nb = 1;
-    if (nb > kFbcMaxBlocks) nb = kFbcMaxBlocks;
+    if (nb > cap) nb = cap;
     return static_cast<int>(nb);
 }
 

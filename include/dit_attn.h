@@ -187,12 +187,30 @@ dit_status dit_attn_q8_workspace_layout(int B, int H, int N, int d, int pv_mode,
  *                  call leaves it zero-filled again.  Calls that share one
  *                  workspace must be ordered (same stream, or synchronised).
  *   Partial sums are fp32 per thread and fp64 across threads and blocks, in a
- *   fixed order: the result is deterministic for a given n.
+ *   fixed order: the result is deterministic for a given n on a given GPU model
+ *   (the grid, at most one wave of resident blocks, follows the SM count).
  */
 size_t fbc_rel_l1_workspace_bytes(int64_t n);
 dit_status fbc_rel_l1(const void* r_cur, const void* r_prev, int64_t n, int dtype,
                       float threshold, double* out_rel, int32_t* out_skip,
                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fbc_rel_l1_sums / fbc_rel_l1_finish — fbc_rel_l1 in two halves, for a
+ * residual sharded across devices (as the token sequence is under the context
+ * parallelism of the ParaAttention page, section "Context Parallelism"):
+ *   fbc_rel_l1_sums   out_sums[0] = Σ|r_cur − r_prev|, out_sums[1] = Σ|r_prev|
+ *                     over this device's n elements (device double[2], 8-byte
+ *                     aligned); arguments and workspace rules as fbc_rel_l1.
+ *   (the caller all-reduces the two doubles, e.g. one NCCL sum)
+ *   fbc_rel_l1_finish rel and skip from the (reduced) sums, with fbc_rel_l1's
+ *                     conventions; sums: device double[2].  One tiny launch.
+ * With one device, sums then finish gives exactly fbc_rel_l1's result.
+ */
+dit_status fbc_rel_l1_sums(const void* r_cur, const void* r_prev, int64_t n, int dtype,
+                           double* out_sums, void* workspace, size_t workspace_bytes, void* stream);
+dit_status fbc_rel_l1_finish(const double* sums, float threshold, double* out_rel, int32_t* out_skip,
+                             void* stream);
 
 /*
  * fbc_rel_l1_noalloc — fbc_rel_l1 without a caller-provided workspace, for

@@ -270,3 +270,14 @@ def test_attn_ex_and_merge_argument_errors(lib):
     assert merge(lparts=[0x71000002, 0x71100000]) == dit.DIT_ERR_INVALID_ARG
     assert merge(o=Q) == dit.DIT_ERR_INVALID_ARG                    # output overwrites a part
     assert merge(lse=0x71000000) == dit.DIT_ERR_INVALID_ARG         # lse overwrites a part's lse
+
+
+def test_fbc_sums_and_finish_argument_errors(lib):
+    ws = lib.fbc_rel_l1_workspace_bytes(64)
+    assert lib.fbc_rel_l1_sums(Q, K, 0, 0, V, O, ws, None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.fbc_rel_l1_sums(Q, K, 64, 0, V + 4, O, ws, None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.fbc_rel_l1_sums(Q, K + 8, 64, 0, V, O, ws, None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.fbc_rel_l1_sums(Q, K, 64, 0, V, O, ws - 1, None) == dit.DIT_ERR_WORKSPACE
+    assert lib.fbc_rel_l1_finish(None, 0.1, V, V + 64, None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.fbc_rel_l1_finish(Q + 4, 0.1, V, V + 64, None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.fbc_rel_l1_finish(Q, float("nan"), V, V + 64, None) == dit.DIT_ERR_INVALID_ARG

@@ -26,6 +26,51 @@ def _global_inputs(B, H, N, d, seed=0):
     return inputs.attn_inputs(inputs.AttnCase("cp", B, H, N, d, seed=seed))
 
 
+def _fbc_worker(rank, world, port, results):
+    import torch.distributed as dist
+
+    import oracle
+    from diffusion_transformer_attention_attn_b200 import context_parallel as cp
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(5)
+        prev = rng.standard_normal(10000).astype(np.float32)
+        cur = (prev + 0.07 * rng.standard_normal(prev.size)).astype(np.float32)
+        cuts = np.linspace(0, prev.size, world + 1).astype(int)
+        a, b = cuts[rank], cuts[rank + 1]
+
+        def sums(c, p):
+            return torch.tensor(oracle.fbc_sums(c.numpy(), p.numpy()), dtype=torch.float64)
+
+        def finish(s, thr):
+            return oracle.rel_from_sums(float(s[0]), float(s[1]), thr)
+        results[rank] = cp.sharded_fbc_rel_l1(torch.from_numpy(cur[a:b]), torch.from_numpy(prev[a:b]), 0.08,
+                                              sums_fn=sums, finish_fn=finish)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_fbc_gives_every_rank_the_whole_residuals_decision():
+    import oracle
+    import torch.multiprocessing as mp
+    world = 3
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_fbc_worker, args=(world, port, results), nprocs=world, join=True, start_method="spawn")
+        res = dict(results)
+    rng = np.random.default_rng(5)
+    prev = rng.standard_normal(10000).astype(np.float32)
+    cur = (prev + 0.07 * rng.standard_normal(prev.size)).astype(np.float32)
+    rel_ref, skip_ref = oracle.fbc_rel_l1(cur, prev, 0.08)
+    for r in range(world):
+        rel, skip = res[r]
+        assert abs(rel - rel_ref) <= 1e-12 * rel_ref and skip == skip_ref
+
+
 def _worker(rank, world, port, scheme, shape, results):
     import torch.distributed as dist
 

@@ -86,3 +86,25 @@ def test_deterministic_and_workspace_reusable():
         assert _gpu_rel(cur, prev, 0.08, ws) == first
     # the ticket counter is back at zero after each call
     assert int(ws[:4].view(torch.int32).item()) == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_sums_then_finish_equals_one_call_and_shards_add_up(dtype):
+    import diffusion_transformer_attention_attn_b200 as dit
+    case = inputs.FbcCase(f"s_{dtype}", 1000, 3072, dtype, 0.05, 0.08, seed=3)
+    cur, prev = inputs.fbc_inputs(case)
+    c, p = _dev(cur).reshape(-1), _dev(prev).reshape(-1)
+    rel1, skip1 = dit.fbc_rel_l1(c, p, 0.08)
+    sums = dit.fbc_rel_l1_sums(c, p)
+    rel2, skip2 = dit.fbc_rel_l1_finish(sums, 0.08)
+    assert rel1.item() == rel2.item() and skip1.item() == skip2.item()
+    num, den = oracle.fbc_sums(cur, prev)
+    s = sums.cpu().numpy()
+    assert abs(s[0] - num) <= FBC_REL_ERR * num and abs(s[1] - den) <= FBC_REL_ERR * den
+    # three shards of the same residual (as three devices would hold it), added on the device
+    n = c.numel()
+    cuts = [0, n // 3, n // 3 + 8, n]
+    total = sum(dit.fbc_rel_l1_sums(c[a:b], p[a:b]) for a, b in zip(cuts[:-1], cuts[1:]))
+    rel3, skip3 = dit.fbc_rel_l1_finish(total.contiguous(), 0.08)
+    rel_ref, skip_ref = oracle.fbc_rel_l1(cur, prev, 0.08)
+    assert abs(rel3.item() - rel_ref) <= FBC_REL_ERR * rel_ref and int(skip3.item()) == skip_ref
