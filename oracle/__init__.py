@@ -298,3 +298,58 @@ def rel_from_sums(num: float, den: float, threshold: float):
     else:
         rel = float("inf") if num > 0 else 0.0
     return rel, int(rel < float(np.float32(threshold)))
+
+
+# ---- 8-bit pre-pass over a token-sharded sequence --------------------------
+# Under Ulysses context parallelism (ParaAttention page, "Context
+# Parallelism"; TMAP image-to-video page, sequence parallelism combined with
+# the 8-bit attention) each device holds a slice of the tokens.  The K mean and
+# the V channel maxima span all tokens, so each device reduces its slice to
+# per-channel sums and maxima, the devices combine them, and each quantises its
+# own tokens with the combined statistics; the 1-byte codes then travel in the
+# all-to-all instead of the bf16 values.
+
+def k_channel_sums(k: np.ndarray) -> np.ndarray:
+    """[B, H, N, d] bf16 bits -> [B, H, d] fp64 sums over the tokens."""
+    return _widen(k).sum(axis=2)
+
+
+def channel_amax(v: np.ndarray) -> np.ndarray:
+    """[B, H, N, d] bf16 bits -> [B, H, d] fp32 max |v| over the tokens."""
+    return np.abs(_widen(v)).max(axis=2).astype(np.float32)
+
+
+def mean_from_sums(sums: np.ndarray, n_total: int) -> np.ndarray:
+    """fp64 sums / N, rounded once to fp32 (the rounding of channel_mean)."""
+    return (np.asarray(sums, dtype=np.float64) / float(n_total)).astype(np.float32)
+
+
+def quant_e4m3_with_amax(x: np.ndarray, amax: np.ndarray):
+    """Per-channel e4m3 codes of x [B,H,N,d] (bf16 bits) with the channel maxima
+    given ([B,H,d] fp32): scale = amax/448 and inv = 448/amax as fp32
+    divisions, code = e4m3(x·inv) (fp32 product); amax = 0 gives zero codes
+    and scales (the zero-scale guard).  Returns (codes, scales)."""
+    amax = np.asarray(amax, dtype=np.float32)
+    with np.errstate(divide="ignore"):
+        scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(0.0)).astype(np.float32)
+        inv = np.where(amax > 0, np.float32(448.0) / amax, np.float32(0.0)).astype(np.float32)
+    xf = _widen(x).astype(np.float32)
+    prod = (xf * inv[:, :, None, :]).astype(np.float32)
+    return e4m3_encode(prod), scale
+
+
+def attention_from_codes(qc, qs, kc, ks, v, vs=None, scale: float | None = None, rows=None) -> np.ndarray:
+    """fp64 attention over dequantised codes: Q = qc·qs (per 128 tokens),
+    K = kc·ks (per 64 tokens), V = e4m3(v)·vs per channel when vs is given,
+    else v as bf16 bits.  The scale defaults to the fp32 1/sqrt(d)."""
+    B, H, N, d = qc.shape
+    tok = np.arange(N)
+    qd = qc.astype(np.float64) * qs[:, :, tok // 128, None].astype(np.float64)
+    kd = kc.astype(np.float64) * ks[:, :, tok // 64, None].astype(np.float64)
+    if vs is not None:
+        vd = e4m3_decode(v).astype(np.float64) * vs[:, :, None, :].astype(np.float64)
+    else:
+        vd = _widen(v)
+    if scale is None:
+        scale = float(np.float32(1.0) / np.sqrt(np.float32(d)))
+    return attention(qd, kd, vd, scale=scale, rows=rows)
