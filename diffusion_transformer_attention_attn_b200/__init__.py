@@ -55,6 +55,9 @@ SIGNATURES = {
     "dit_attn_fwd_q8": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p, _f, _i, _i, _p, _sz, _p]),
     "dit_attn_q8_quantize": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _i, _i, _p, _sz, _p]),
     "dit_attn_q8_workspace_layout": (_i, [_i, _i, _i, _i, _i, _p]),
+    "dit_attn_q8_channel_stats": (_i, [_p, _p, _i, _i, _i, _i, _p, _i, _i, _p, _p, _p, _sz, _p]),
+    "dit_attn_q8_quantize_global": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _i, _i, _p, _p, _i64, _p, _sz, _p]),
+    "dit_attn_fwd_q8_prequantized": (_i, [_p, _sz, _p, _p, _i, _i, _i, _i, _p, _f, _i, _p]),
     "fbc_rel_l1_workspace_bytes": (_sz, [_i64]),
     "fbc_rel_l1": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p, _sz, _p]),
     "fbc_rel_l1_noalloc": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p]),
@@ -121,6 +124,12 @@ def _check(status: int, what: str):
         raise DitError(status, what)
 
 
+def _same_layout(a, b) -> bool:
+    """Same shape, and the same strides in every dimension longer than 1 (the
+    stride of a length-1 dimension never addresses anything)."""
+    return a.shape == b.shape and all(x == y or n == 1 for x, y, n in zip(a.stride(), b.stride(), a.shape))
+
+
 def _attn_strides(t):
     """(b, h, n) element strides of a [B, H, N, d] tensor with unit d stride."""
     if t.dim() != 4 or t.stride(3) != 1:
@@ -140,7 +149,7 @@ def dit_attn_fwd(q, k, v, o=None, scale: float | None = None, stream=None):
     for t in (q, k, v, o):
         if t.dtype != torch.bfloat16 or not t.is_cuda:
             raise TypeError("dit_attn_fwd expects bf16 CUDA tensors")
-        if t.shape != q.shape or t.stride() != q.stride():
+        if not _same_layout(t, q):
             raise ValueError("q, k, v, o must share shape and strides")
     B, H, N, d = q.shape
     st = lib.dit_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), B, H, N, d,
@@ -163,9 +172,9 @@ def dit_attn_fwd_ex(q, k, v, o=None, lse=None, scale: float | None = None, strea
     for t in (q, k, v, o):
         if t.dtype != torch.bfloat16 or not t.is_cuda:
             raise TypeError("dit_attn_fwd_ex expects bf16 CUDA tensors")
-    if o.shape != q.shape or o.stride() != q.stride():
+    if not _same_layout(o, q):
         raise ValueError("q and o must share shape and strides")
-    if v.shape != k.shape or v.stride() != k.stride():
+    if not _same_layout(v, k):
         raise ValueError("k and v must share shape and strides")
     B, H, Nq, d = q.shape
     if k.shape[0] != B or k.shape[1] != H or k.shape[3] != d:
@@ -193,7 +202,7 @@ def dit_attn_merge(o_parts, lse_parts, o=None, lse=None, stream=None):
         raise ValueError("need as many log-sum-exps as outputs, at least one")
     ref = o_parts[0]
     for t in o_parts:
-        if t.dtype != torch.bfloat16 or t.shape != ref.shape or t.stride() != ref.stride():
+        if t.dtype != torch.bfloat16 or not _same_layout(t, ref):
             raise ValueError("o_parts must be bf16 tensors of one shape and stride")
     B, H, N, d = ref.shape
     for t in lse_parts:
@@ -201,7 +210,7 @@ def dit_attn_merge(o_parts, lse_parts, o=None, lse=None, stream=None):
             raise ValueError("lse_parts must be contiguous fp32 tensors of B*H*N elements")
     if o is None:
         o = torch.empty_like(ref)
-    if o.shape != ref.shape or o.stride() != ref.stride():
+    if not _same_layout(o, ref):
         raise ValueError("o must share the parts' shape and strides")
     if lse is True:
         lse = torch.empty(B, H, N, dtype=torch.float32, device=ref.device)
@@ -267,7 +276,7 @@ def _check_attn_tensors(q, k, v, o):
     for t in (q, k, v) + ((o,) if o is not None else ()):
         if t.dtype != torch.bfloat16 or not t.is_cuda:
             raise TypeError("expected bf16 CUDA tensors")
-        if t.shape != q.shape or t.stride() != q.stride():
+        if not _same_layout(t, q):
             raise ValueError("q, k, v, o must share shape and strides")
 
 
@@ -303,6 +312,63 @@ def dit_attn_q8_quantize(q, k, v, smooth_k: bool = True, pv_mode="fp8", workspac
                                   _stream_ptr(stream))
     _check(st, "dit_attn_q8_quantize")
     return workspace
+
+
+def dit_attn_q8_channel_stats(k, v, smooth_k: bool = True, pv_mode="fp8", k_sum=None, v_amax=None, workspace=None,
+                              stream=None):
+    """Per-channel K sums (float64 [B,H,d]) and V maxima (float32 [B,H,d])
+    over this slice of the tokens, for the devices of a Ulysses group to
+    combine (sum, max).  Returns (k_sum, v_amax)."""
+    import torch
+    lib = load_library()
+    _check_attn_tensors(k, k, v, None)
+    B, H, N, d = k.shape
+    if k_sum is None:
+        k_sum = torch.empty(B, H, d, dtype=torch.float64, device=k.device)
+    if v_amax is None:
+        v_amax = torch.empty(B, H, d, dtype=torch.float32, device=k.device)
+    if workspace is None:
+        workspace = q8_workspace(B, H, N, d, pv_mode, k.device)
+    st = lib.dit_attn_q8_channel_stats(k.data_ptr(), v.data_ptr(), B, H, N, d, _attn_strides(k), int(bool(smooth_k)),
+                                       _pv(pv_mode), k_sum.data_ptr(), v_amax.data_ptr(), workspace.data_ptr(),
+                                       workspace.numel(), _stream_ptr(stream))
+    _check(st, "dit_attn_q8_channel_stats")
+    return k_sum, v_amax
+
+
+def dit_attn_q8_quantize_global(q, k, v, k_sum, v_amax, n_total: int, smooth_k: bool = True, pv_mode="fp8",
+                                workspace=None, stream=None):
+    """Quantise this slice of the tokens with statistics combined over all
+    n_total tokens; returns the workspace (codes and scales)."""
+    lib = load_library()
+    _check_attn_tensors(q, k, v, None)
+    B, H, N, d = q.shape
+    if workspace is None:
+        workspace = q8_workspace(B, H, N, d, pv_mode, q.device)
+    st = lib.dit_attn_q8_quantize_global(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, _attn_strides(q),
+                                         int(bool(smooth_k)), _pv(pv_mode), k_sum.data_ptr(), v_amax.data_ptr(),
+                                         int(n_total), workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(st, "dit_attn_q8_quantize_global")
+    return workspace
+
+
+def dit_attn_fwd_q8_prequantized(workspace, B: int, H: int, N: int, o=None, v=None, scale: float | None = None,
+                                 pv_mode="fp8", d: int = 128, stream=None):
+    """The 8-bit attention kernel alone, on a workspace whose codes and scales
+    the caller filled (layout of dit_attn_q8_workspace_layout for B, H, N).
+    v: the bf16 V in bf16-PV mode.  Returns o (bf16 [B, H, N, d])."""
+    import torch
+    lib = load_library()
+    if o is None:
+        o = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=workspace.device)
+    if v is not None and not _same_layout(v, o):
+        raise ValueError("v and o must share shape and strides")
+    st = lib.dit_attn_fwd_q8_prequantized(workspace.data_ptr(), workspace.numel(),
+                                          v.data_ptr() if v is not None else None, o.data_ptr(), B, H, N, d,
+                                          _attn_strides(o), float(scale) if scale else 0.0, _pv(pv_mode),
+                                          _stream_ptr(stream))
+    _check(st, "dit_attn_fwd_q8_prequantized")
+    return o
 
 
 def fbc_rel_l1_workspace_bytes(n: int) -> int:

@@ -14,6 +14,12 @@ work), and the cache decision over a sharded residual:
   around the ring; every step attends the local queries to the chunk in hand
   (``dit_attn_fwd_ex`` with log-sum-exp), while the next chunk is already in
   flight, and the per-chunk results are merged (``dit_attn_merge``).
+* ``ulysses_attention_q8`` — Ulysses with the 8-bit attention, the all-to-all
+  moving 1-byte codes: each rank reduces its tokens to per-channel K sums and
+  V maxima (``dit_attn_q8_channel_stats``), two all-reduces combine them, each
+  rank quantises its own tokens (``dit_attn_q8_quantize_global``), the codes
+  and block scales travel to the head-sharded layout, and the attention runs
+  on them (``dit_attn_fwd_q8_prequantized``).
 * ``sharded_fbc_rel_l1`` — the first-block-cache difference of a residual
   sharded like the sequence: each rank reduces its slice to two sums
   (``fbc_rel_l1_sums``), one all-reduce adds them, and ``fbc_rel_l1_finish``
@@ -21,7 +27,8 @@ work), and the cache decision over a sharded residual:
 
 The collectives are torch.distributed calls (NCCL between GPUs); the attention,
 the merge and the reductions are the library's kernels.  ``attn_fn``,
-``attn_lse_fn``, ``merge_fn``, ``sums_fn`` and ``finish_fn`` may be replaced,
+``attn_lse_fn``, ``merge_fn``, ``stats_fn``, ``quant_fn``, ``codes_attn_fn``,
+``sums_fn`` and ``finish_fn`` may be replaced,
 e.g. to run the data movement on CPU ranks.
 """
 from __future__ import annotations
@@ -155,3 +162,71 @@ def sharded_fbc_rel_l1(r_cur, r_prev, threshold: float, group=None, sums_fn=None
     if world > 1:
         dist.all_reduce(sums, op=dist.ReduceOp.SUM, group=group)
     return (finish_fn or _default_finish)(sums, threshold)
+
+
+# ---- Ulysses with 8-bit transport --------------------------------------------
+
+CODE_KEYS = ("q_codes", "k_codes", "v_codes")
+
+
+def _default_stats(k, v, smooth_k, pv_mode):
+    from . import dit_attn_q8_channel_stats
+    return dit_attn_q8_channel_stats(k, v, smooth_k=smooth_k, pv_mode=pv_mode)
+
+
+def _default_quant(q, k, v, k_sum, v_amax, n_total, smooth_k, pv_mode):
+    from . import dit_attn_q8_quantize_global, q8_views
+    B, H, N, d = q.shape
+    ws = dit_attn_q8_quantize_global(q, k, v, k_sum, v_amax, n_total, smooth_k=smooth_k, pv_mode=pv_mode)
+    return q8_views(ws, B, H, N, d, pv_mode)
+
+
+def _default_codes_attn(parts, v, pv_mode):
+    """parts: head-sharded codes and scales (q8_views names)."""
+    from . import dit_attn_fwd_q8_prequantized, q8_views, q8_workspace
+    B, H, N, d = parts["q_codes"].shape
+    ws = q8_workspace(B, H, N, d, pv_mode, parts["q_codes"].device)
+    dst = q8_views(ws, B, H, N, d, pv_mode)
+    for name, t in parts.items():
+        dst[name].copy_(t)
+    return dit_attn_fwd_q8_prequantized(ws, B, H, N, v=v, pv_mode=pv_mode, d=d)
+
+
+def ulysses_attention_q8(q, k, v, group=None, smooth_k: bool = True, pv_mode="fp8", stats_fn=None, quant_fn=None,
+                         codes_attn_fn=None):
+    """8-bit attention over the full sequence from sequence-sharded
+    [B, H, N/P, d] q, k, v, with the all-to-all carrying the 8-bit codes
+    (bf16 V instead in bf16-PV mode).  N/P must be a multiple of 128 (whole
+    Q blocks per rank).  Returns this rank's [B, H, N/P, d] output."""
+    import torch
+    import torch.distributed as dist
+    world, rank = _group_info(group)
+    B, H, Nl, d = q.shape
+    if H % world:
+        raise ValueError(f"{H} heads do not split over {world} ranks")
+    if Nl % 128:
+        raise ValueError("each rank must hold whole 128-token blocks")
+    fp8 = pv_mode in ("fp8", 0)
+    k_sum, v_amax = (stats_fn or _default_stats)(k, v, smooth_k, pv_mode)
+    if world > 1:
+        dist.all_reduce(k_sum, op=dist.ReduceOp.SUM, group=group)
+        dist.all_reduce(v_amax, op=dist.ReduceOp.MAX, group=group)
+    local = (quant_fn or _default_quant)(q, k, v, k_sum, v_amax, Nl * world, smooth_k, pv_mode)
+    hp = H // world
+    names = [n for n in CODE_KEYS if n in local]
+    parts = {}
+    if world > 1:
+        # 1-byte codes travel as 32-bit words (d is a multiple of 4).
+        moved = seq_to_heads([local[n].contiguous().view(torch.int32) for n in names], world, group)
+        for n, t in zip(names, moved):
+            parts[n] = t.contiguous().view(local[n].dtype)
+        for n in ("q_scale", "k_scale"):
+            parts[n] = seq_to_heads([local[n].unsqueeze(-1)], world, group)[0].squeeze(-1).contiguous()
+        vh = None if fp8 else seq_to_heads([v], world, group)[0].contiguous()
+    else:
+        parts = {n: local[n] for n in names + ["q_scale", "k_scale"]}
+        vh = None if fp8 else v
+    if fp8:
+        parts["v_scale"] = local["v_scale"][:, rank * hp:(rank + 1) * hp].contiguous()
+    oh = (codes_attn_fn or _default_codes_attn)(parts, vh, pv_mode)
+    return oh if world == 1 else heads_to_seq(oh, world, group)

@@ -320,6 +320,89 @@ dit_status dit_attn_q8_quantize(const void* q, const void* k, const void* v, int
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
+// ---- token-sharded 8-bit pre-pass and attention from codes ----------------
+
+namespace {
+bool overlap_bytes(const void* a, int64_t na, const void* b, int64_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + static_cast<uintptr_t>(nb) && y < x + static_cast<uintptr_t>(na);
+}
+}  // namespace
+
+dit_status dit_attn_q8_channel_stats(const void* k, const void* v, int B, int H, int N, int d, const int64_t* strides,
+                                     int smooth_k, int pv_mode, double* k_sum, float* v_amax, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    int64_t sb, sh, sn;
+    dit_status st = check_attn_args(k, k, v, nullptr, B, H, N, d, strides, &sb, &sh, &sn, false);
+    if (st != DIT_OK) return st;
+    if ((st = check_q8_args(d, smooth_k, pv_mode, workspace, workspace_bytes, B, H, N)) != DIT_OK) return st;
+    if (!k_sum || !v_amax || (reinterpret_cast<uintptr_t>(k_sum) & 7u) || (reinterpret_cast<uintptr_t>(v_amax) & 3u))
+        return DIT_ERR_INVALID_ARG;
+    const int64_t nstat = static_cast<int64_t>(B) * H * d;
+    const int64_t wsz = static_cast<int64_t>(q8_layout(B, H, N, d, pv_mode == DIT_PV_FP8_E4M3).total);
+    if (overlap_bytes(k_sum, nstat * 8, workspace, wsz) || overlap_bytes(v_amax, nstat * 4, workspace, wsz) ||
+        overlap_bytes(k_sum, nstat * 8, v_amax, nstat * 4))
+        return DIT_ERR_INVALID_ARG;
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    cudaError_t e = launch_q8_slice_stats(k, v, sb, sh, sn, B, H, N, smooth_k, pv_mode == DIT_PV_FP8_E4M3,
+                                          static_cast<uint8_t*>(workspace), k_sum, v_amax,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+dit_status dit_attn_q8_quantize_global(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                                       const int64_t* strides, int smooth_k, int pv_mode, const double* k_sum,
+                                       const float* v_amax, int64_t n_total, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+    int64_t sb, sh, sn;
+    dit_status st = check_attn_args(q, k, v, nullptr, B, H, N, d, strides, &sb, &sh, &sn, false);
+    if (st != DIT_OK) return st;
+    if ((st = check_q8_args(d, smooth_k, pv_mode, workspace, workspace_bytes, B, H, N)) != DIT_OK) return st;
+    if (!k_sum || !v_amax || (reinterpret_cast<uintptr_t>(k_sum) & 7u) || (reinterpret_cast<uintptr_t>(v_amax) & 3u))
+        return DIT_ERR_INVALID_ARG;
+    if (n_total < N) return DIT_ERR_INVALID_ARG;
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    cudaError_t e = launch_q8_quantize_global(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_mode == DIT_PV_FP8_E4M3,
+                                              k_sum, v_amax, n_total, static_cast<uint8_t*>(workspace),
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+dit_status dit_attn_fwd_q8_prequantized(const void* workspace, size_t workspace_bytes, const void* v, void* o, int B,
+                                        int H, int N, int d, const int64_t* strides, float scale, int pv_mode,
+                                        void* stream) {
+    if (pv_mode != DIT_PV_FP8_E4M3 && pv_mode != DIT_PV_BF16) return DIT_ERR_INVALID_ARG;
+    const int pv_fp8 = pv_mode == DIT_PV_FP8_E4M3;
+    const void* vv = pv_fp8 ? o : v;  // stands in for V during validation in FP8 mode
+    int64_t sb, sh, sn;
+    dit_status st = check_attn_args(o, o, vv, nullptr, B, H, N, d, strides, &sb, &sh, &sn, false);
+    if (st != DIT_OK) return st;
+    if (!(scale == scale) || std::isinf(scale)) return DIT_ERR_INVALID_ARG;
+    if ((st = check_q8_args(d, 0, pv_mode, workspace, workspace_bytes, B, H, N)) != DIT_OK) return st;
+    const Q8Layout L = q8_layout(B, H, N, d, pv_fp8);
+    const int64_t span = ((B - 1) * sb + (H - 1) * sh + (N - 1) * sn + d) * 2;
+    if (overlap_bytes(o, span, workspace, static_cast<int64_t>(L.total))) return DIT_ERR_WORKSPACE;
+    if (!pv_fp8 && overlap_bytes(o, span, v, span)) return DIT_ERR_INVALID_ARG;
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+    CUtensorMap tq8, tk8, tv;
+    if ((st = encode_u8_map(&tq8, ws + L.q_codes, B, H, N)) != DIT_OK) return st;
+    if ((st = encode_u8_map(&tk8, ws + L.k_codes, B, H, N)) != DIT_OK) return st;
+    if (pv_fp8)
+        st = encode_u8_map(&tv, ws + L.v_codes, B, H, N);
+    else
+        st = encode_bf16_map(&tv, v, B, H, N, d, sb, sh, sn);
+    if (st != DIT_OK) return st;
+    const float sc = scale > 0.f ? scale : default_scale(d);
+    const float scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
+    cudaError_t e = launch_attn_q8(tq8, tk8, tv, pv_fp8, ws, L, o, sb, sh, sn, B, H, N, scale_log2, ds->err_word,
+                                   static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
 dit_status dit_attn_fwd_q8(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
                            const int64_t* strides, float scale, int smooth_k, int pv_mode, void* workspace,
                            size_t workspace_bytes, void* stream) {

@@ -48,6 +48,19 @@ Q8Layout q8_layout(int B, int H, int N, int d, int pv_fp8);
 cudaError_t launch_q8_prepass(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
                               int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream);
 
+// The quantisation launches of the pre-pass alone (K mean and V scales
+// already in `ws`).
+cudaError_t launch_q8_codes(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
+                            int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream);
+// Token-sharded pre-pass: the slice's per-channel K sums (fp64) and V maxima,
+// then quantisation with the statistics combined over n_total tokens.
+cudaError_t launch_q8_slice_stats(const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H,
+                                  int N, int smooth_k, int pv_fp8, uint8_t* ws, double* k_sum, float* v_amax,
+                                  cudaStream_t stream);
+cudaError_t launch_q8_quantize_global(const void* q, const void* k, const void* v, int64_t sb, int64_t sh,
+                                      int64_t sn, int B, int H, int N, int smooth_k, int pv_fp8, const double* k_sum,
+                                      const float* v_amax, int64_t n_total, uint8_t* ws, cudaStream_t stream);
+
 // 8-bit attention over the pre-pass products.  tq8/tk8: 4-D maps over the
 // INT8 codes {d, N, H, B}, box {128, 128, 1, 1}; tv: e4m3 codes (same box,
 // pv_fp8) or the caller's bf16 V (box {64, 128, 1, 1}).

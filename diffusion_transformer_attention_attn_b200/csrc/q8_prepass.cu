@@ -14,6 +14,12 @@
 //   * V (FP8 PV only): per channel, amax over all N tokens, scale = amax/448,
 //     code = e4m3(x·448/amax), round to nearest even, saturating; same guard.
 //
+// Token-sharded form (launch_q8_slice_stats, launch_q8_quantize_global): each
+// device reduces its token slice to per-channel K sums and V maxima, the
+// devices combine them (sum, max), and each quantises its own tokens with the
+// combined statistics, so that the 1-byte codes, not the bf16 values, travel
+// in a Ulysses all-to-all.
+//
 // Three launches, each HBM-bound with 16-byte vector loads:
 //   q8_stats_kernel     per (b,h) and chunk of 256 tokens: fp64 column sums of
 //                       K and column |V| maxima -> partials
@@ -227,6 +233,45 @@ __global__ void __launch_bounds__(kQuantThreads)
     }
 }
 
+// Token-sharded form (one slice of the tokens per device): the per-channel
+// K sums and V maxima of this slice, for the devices to combine.  grid B*H,
+// 128 threads (one per channel); the same fixed-order sum as q8_finalize.
+__global__ void q8_slice_stats_kernel(const double* __restrict__ psum, const float* __restrict__ pmax, int n_chunks,
+                                      int want_sum, int want_vmax, double* __restrict__ k_sum,
+                                      float* __restrict__ v_amax) {
+    constexpr int D = 128;
+    const int bh = blockIdx.x, c = threadIdx.x;
+    double s = 0.0;
+    float m = 0.f;
+    for (int i = 0; i < n_chunks; ++i) {
+        const int64_t idx = (static_cast<int64_t>(bh) * n_chunks + i) * D + c;
+        if (want_sum) s += psum[idx];
+        if (want_vmax) m = fmaxf(m, pmax[idx]);
+    }
+    k_sum[bh * D + c] = s;
+    v_amax[bh * D + c] = m;
+}
+
+// The K mean and V scales from the combined statistics of all slices
+// (n_total tokens): the arithmetic of q8_finalize_kernel.
+__global__ void q8_finalize_global_kernel(const double* __restrict__ k_sum, const float* __restrict__ v_amax,
+                                          int64_t n_total, int want_sum, int want_vmax, float* __restrict__ k_mean,
+                                          float* __restrict__ v_scale, float* __restrict__ v_inv) {
+    constexpr int D = 128;
+    const int bh = blockIdx.x, c = threadIdx.x;
+    k_mean[bh * D + c] = want_sum ? static_cast<float>(k_sum[bh * D + c] / static_cast<double>(n_total)) : 0.f;
+    if (want_vmax) {
+        const float m = v_amax[bh * D + c];
+        float sc = 0.f, inv = 0.f;
+        if (m > 0.f) {  // zero-scale guard
+            sc = __fdiv_rn(m, 448.f);
+            inv = __fdiv_rn(448.f, m);
+        }
+        v_scale[bh * D + c] = sc;
+        v_inv[bh * D + c] = inv;
+    }
+}
+
 }  // namespace
 
 Q8Layout q8_layout(int B, int H, int N, int d, int pv_fp8) {
@@ -253,18 +298,27 @@ Q8Layout q8_layout(int B, int H, int N, int d, int pv_fp8) {
 cudaError_t launch_q8_prepass(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
                               int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
     const Q8Layout L = q8_layout(B, H, N, 128, pv_fp8);
-    const int BH = B * H;
     double* psum = reinterpret_cast<double*>(ws + L.psum);
     float* pmax = reinterpret_cast<float*>(ws + L.pmax);
     float* k_mean = reinterpret_cast<float*>(ws + L.k_mean);
     float* v_scale = reinterpret_cast<float*>(ws + L.v_scale);
     float* v_inv = reinterpret_cast<float*>(ws + L.v_inv);
+    const int BH = B * H;
     if (smooth_k || pv_fp8) {
         q8_stats_kernel<<<dim3(L.n_chunks, BH), kStatThreads, 0, stream>>>(k, v, sb, sh, sn, H, N, kQ8StatChunk,
                                                                            smooth_k, pv_fp8, psum, pmax);
         q8_finalize_kernel<<<BH, 128, 0, stream>>>(psum, pmax, L.n_chunks, N, smooth_k, pv_fp8, k_mean, v_scale,
                                                    v_inv);
     }
+    return launch_q8_codes(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, stream);
+}
+
+cudaError_t launch_q8_codes(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
+                            int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
+    const Q8Layout L = q8_layout(B, H, N, 128, pv_fp8);
+    const int BH = B * H;
+    const float* k_mean = reinterpret_cast<const float*>(ws + L.k_mean);
+    const float* v_inv = reinterpret_cast<const float*>(ws + L.v_inv);
     q8_quant_int8_kernel<128><<<dim3((N + 127) / 128, BH), kQuantThreads, 0, stream>>>(
         q, sb, sh, sn, H, N, nullptr, reinterpret_cast<int8_t*>(ws + L.q_codes),
         reinterpret_cast<float*>(ws + L.q_scale));
@@ -275,6 +329,33 @@ cudaError_t launch_q8_prepass(const void* q, const void* k, const void* v, int64
         q8_quant_e4m3_kernel<<<dim3((N + 127) / 128, BH), kQuantThreads, 0, stream>>>(
             v, sb, sh, sn, H, N, v_inv, ws + L.v_codes);
     return cudaGetLastError();
+}
+
+cudaError_t launch_q8_slice_stats(const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H,
+                                  int N, int smooth_k, int pv_fp8, uint8_t* ws, double* k_sum, float* v_amax,
+                                  cudaStream_t stream) {
+    const Q8Layout L = q8_layout(B, H, N, 128, pv_fp8);
+    const int BH = B * H;
+    double* psum = reinterpret_cast<double*>(ws + L.psum);
+    float* pmax = reinterpret_cast<float*>(ws + L.pmax);
+    if (smooth_k || pv_fp8)
+        q8_stats_kernel<<<dim3(L.n_chunks, BH), kStatThreads, 0, stream>>>(k, v, sb, sh, sn, H, N, kQ8StatChunk,
+                                                                           smooth_k, pv_fp8, psum, pmax);
+    q8_slice_stats_kernel<<<BH, 128, 0, stream>>>(psum, pmax, L.n_chunks, smooth_k, pv_fp8, k_sum, v_amax);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_q8_quantize_global(const void* q, const void* k, const void* v, int64_t sb, int64_t sh,
+                                      int64_t sn, int B, int H, int N, int smooth_k, int pv_fp8, const double* k_sum,
+                                      const float* v_amax, int64_t n_total, uint8_t* ws, cudaStream_t stream) {
+    const Q8Layout L = q8_layout(B, H, N, 128, pv_fp8);
+    q8_finalize_global_kernel<<<B * H, 128, 0, stream>>>(k_sum, v_amax, n_total, smooth_k, pv_fp8,
+                                                         reinterpret_cast<float*>(ws + L.k_mean),
+                                                         reinterpret_cast<float*>(ws + L.v_scale),
+                                                         reinterpret_cast<float*>(ws + L.v_inv));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_q8_codes(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, stream);
 }
 
 }  // namespace ditk

@@ -167,6 +167,44 @@ dit_status dit_attn_q8_quantize(const void* q, const void* k, const void* v,
 dit_status dit_attn_q8_workspace_layout(int B, int H, int N, int d, int pv_mode, size_t* offsets);
 
 /*
+ * Token-sharded 8-bit path (Ulysses context parallelism with 8-bit attention).
+ *
+ * Defined by: "ParaAttention" (diffusers docs), section "Context Parallelism",
+ * and the TMAP image-to-video blog, where sequence parallelism (Ulysses, the
+ * all-to-all overlapped with computation) is combined with 8-bit attention.
+ * Each device holds a slice of the tokens of every head.  The K channel mean
+ * and the V channel maxima span all tokens, so:
+ *   1. dit_attn_q8_channel_stats: this slice's per-channel K sums (fp64,
+ *      zero when smooth_k = 0) and V maxima (fp32, zero in bf16-PV mode),
+ *      both [B, H, d] device arrays; the devices then add the sums and take
+ *      the maximum of the maxima (e.g. two all-reduces);
+ *   2. dit_attn_q8_quantize_global: writes this slice's codes and scales into
+ *      the workspace (layout of dit_attn_q8_workspace_layout for the slice's N
+ *      tokens) with the K mean = k_sum / n_total and V scales = v_amax / 448;
+ *   3. the caller moves codes and scales in the all-to-all (1 byte per value
+ *      instead of 2) into a workspace laid out for H' heads and all N tokens,
+ *      with the V scales of those heads;
+ *   4. dit_attn_fwd_q8_prequantized: the attention kernel alone on that
+ *      workspace (v: the bf16 V [B, H', N, d] in bf16-PV mode, else unused
+ *      and may be NULL; o and v share `strides`).
+ * When every slice holds whole 128-token blocks, the codes equal those that
+ * dit_attn_fwd_q8 writes for the whole sequence, and so does the output.
+ * Arguments, alignment and errors as dit_attn_q8_quantize / dit_attn_fwd_q8;
+ * n_total >= N.
+ */
+dit_status dit_attn_q8_channel_stats(const void* k, const void* v, int B, int H, int N, int d,
+                                     const int64_t* strides, int smooth_k, int pv_mode,
+                                     double* k_sum, float* v_amax,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+dit_status dit_attn_q8_quantize_global(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                                       const int64_t* strides, int smooth_k, int pv_mode,
+                                       const double* k_sum, const float* v_amax, int64_t n_total,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+dit_status dit_attn_fwd_q8_prequantized(const void* workspace, size_t workspace_bytes, const void* v, void* o,
+                                        int B, int H, int N, int d, const int64_t* strides, float scale,
+                                        int pv_mode, void* stream);
+
+/*
  * fbc_rel_l1 — first-block-cache residual difference and decision:
  *   rel  = Σ|r_cur − r_prev| / Σ|r_prev|   (over all n elements)
  *   skip = rel < threshold                 (1: reuse the cached residual)

@@ -281,3 +281,30 @@ def test_fbc_sums_and_finish_argument_errors(lib):
     assert lib.fbc_rel_l1_finish(None, 0.1, V, V + 64, None) == dit.DIT_ERR_INVALID_ARG
     assert lib.fbc_rel_l1_finish(Q + 4, 0.1, V, V + 64, None) == dit.DIT_ERR_INVALID_ARG
     assert lib.fbc_rel_l1_finish(Q, float("nan"), V, V + 64, None) == dit.DIT_ERR_INVALID_ARG
+
+
+def test_sharded_q8_argument_errors(lib):
+    wsb = lib.dit_attn_q8_workspace_bytes(1, 2, 256, 128, 0)
+    KS, VA = 0x62000000, 0x63000000
+    st = lambda **kw: lib.dit_attn_q8_channel_stats(kw.get("k", K), kw.get("v", V), 1, 2, 256, kw.get("d", 128), None,
+                                                    kw.get("smooth", 1), kw.get("mode", 0), kw.get("ks", KS),
+                                                    kw.get("va", VA), kw.get("ws", WS), kw.get("wsb", wsb), None)
+    assert st(k=0) == dit.DIT_ERR_INVALID_ARG
+    assert st(d=64) == dit.DIT_ERR_UNSUPPORTED
+    assert st(mode=3) == dit.DIT_ERR_INVALID_ARG
+    assert st(ks=0) == dit.DIT_ERR_INVALID_ARG
+    assert st(ks=KS + 4) == dit.DIT_ERR_INVALID_ARG
+    assert st(va=WS + 256) == dit.DIT_ERR_INVALID_ARG             # inside the workspace
+    assert st(wsb=16) == dit.DIT_ERR_WORKSPACE
+    qg = lambda **kw: lib.dit_attn_q8_quantize_global(Q, K, V, 1, 2, 256, 128, None, 1, 0, kw.get("ks", KS), VA,
+                                                      kw.get("n", 512), WS, wsb, None)
+    assert qg(n=100) == dit.DIT_ERR_INVALID_ARG                   # n_total below this slice's tokens
+    assert qg(ks=0) == dit.DIT_ERR_INVALID_ARG
+    pq = lambda **kw: lib.dit_attn_fwd_q8_prequantized(kw.get("ws", WS), kw.get("wsb", wsb), kw.get("v", None),
+                                                       kw.get("o", O), 1, 2, 256, 128, None, kw.get("scale", 0.0),
+                                                       kw.get("mode", 0), None)
+    assert pq(o=0) == dit.DIT_ERR_INVALID_ARG
+    assert pq(mode=1) == dit.DIT_ERR_INVALID_ARG                  # bf16 PV needs V
+    assert pq(scale=float("nan")) == dit.DIT_ERR_INVALID_ARG
+    assert pq(wsb=1) == dit.DIT_ERR_WORKSPACE
+    assert pq(ws=WS + 128) == dit.DIT_ERR_WORKSPACE

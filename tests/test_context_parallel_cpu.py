@@ -160,3 +160,77 @@ def test_world_of_one_runs_locally():
         assert torch.equal(out, x + 1)
     finally:
         dist.destroy_process_group()
+
+
+def _q8_worker(rank, world, port, shape, pv_mode, smooth_k, results):
+    import torch.distributed as dist
+
+    import oracle
+    from diffusion_transformer_attention_attn_b200 import context_parallel as cp
+    from diffusion_transformer_attention_attn_b200 import inputs
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, H, N, d = shape
+        q, k, v = inputs.attn_inputs(inputs.AttnCase("cpq8", B, H, N, d, k_offset_std=3.0))
+        Nl = N // world
+        sl = slice(rank * Nl, (rank + 1) * Nl)
+        tq, tk, tv = (torch.from_numpy(inputs.bf16_to_f32(np.ascontiguousarray(x[:, :, sl]))) for x in (q, k, v))
+
+        def bits(t):
+            return inputs.bf16_bits(t.contiguous().numpy())
+
+        def stats(k_, v_, smooth, mode):
+            ks = oracle.k_channel_sums(bits(k_)) if smooth else np.zeros(k_.shape[:2] + (d,))
+            va = oracle.channel_amax(bits(v_)) if mode == "fp8" else np.zeros(v_.shape[:2] + (d,), np.float32)
+            return torch.from_numpy(ks), torch.from_numpy(va)
+
+        def quant(q_, k_, v_, k_sum, v_amax, n_total, smooth, mode):
+            qc, qs = oracle.quant_int8_blocks(bits(q_), 128)
+            mean = oracle.mean_from_sums(k_sum.numpy(), n_total) if smooth else None
+            kc, ks = oracle.quant_int8_blocks(bits(k_), 64, mean)
+            out = {"q_codes": qc, "q_scale": qs, "k_codes": kc, "k_scale": ks}
+            if mode == "fp8":
+                out["v_codes"], out["v_scale"] = oracle.quant_e4m3_with_amax(bits(v_), v_amax.numpy())
+            return {n: torch.from_numpy(np.ascontiguousarray(a)) for n, a in out.items()}
+
+        def codes_attn(parts, vh, mode):
+            p = {n: t.numpy() for n, t in parts.items()}
+            if mode == "fp8":
+                o = oracle.attention_from_codes(p["q_codes"], p["q_scale"], p["k_codes"], p["k_scale"],
+                                                p["v_codes"], p["v_scale"])
+            else:
+                o = oracle.attention_from_codes(p["q_codes"], p["q_scale"], p["k_codes"], p["k_scale"], bits(vh))
+            return torch.from_numpy(o)
+        out = cp.ulysses_attention_q8(tq, tk, tv, smooth_k=smooth_k, pv_mode=pv_mode, stats_fn=stats, quant_fn=quant,
+                                      codes_attn_fn=codes_attn)
+        results[rank] = out.numpy()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,pv_mode,smooth_k", [(2, "fp8", True), (4, "fp8", False), (2, "bf16", True)])
+def test_ulysses_q8_moves_codes_and_matches_the_single_device_codes(world, pv_mode, smooth_k):
+    import oracle
+    import torch.multiprocessing as mp
+    from diffusion_transformer_attention_attn_b200 import inputs
+    shape = (1, 4, 1024, 128)
+    B, H, N, d = shape
+    q, k, v = inputs.attn_inputs(inputs.AttnCase("cpq8", B, H, N, d, k_offset_std=3.0))
+    qc, qs = oracle.quant_int8_blocks(q, 128)
+    kc, ks = oracle.quant_int8_blocks(k, 64, oracle.channel_mean(k) if smooth_k else None)
+    if pv_mode == "fp8":
+        vc, vs = oracle.quant_e4m3_channels(v)
+        ref = oracle.attention_from_codes(qc, qs, kc, ks, vc, vs)
+    else:
+        ref = oracle.attention_from_codes(qc, qs, kc, ks, v)
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_q8_worker, args=(world, port, shape, pv_mode, smooth_k, results), nprocs=world,
+                           join=True, start_method="spawn")
+        res = dict(results)
+    got = np.concatenate([res[r] for r in range(world)], axis=2)
+    assert np.array_equal(got, ref)
