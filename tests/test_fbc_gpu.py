@@ -47,7 +47,7 @@ def _check(cur, prev, thr):
     return rel
 
 
-@pytest.mark.parametrize("case", [inputs.FBC_TINY, inputs.FBC_IMAGE])
+@pytest.mark.parametrize("case", [inputs.FBC_TINY, inputs.FBC_IMAGE, inputs.FBC_VIDEO_LONG], ids=lambda c: c.name)
 def test_workloads(case):
     cur, prev = inputs.fbc_inputs(case)
     _check(cur, prev, case.threshold)

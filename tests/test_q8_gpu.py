@@ -194,3 +194,17 @@ def test_video_mid_workload_sampled_rows():
         out = from_device_bf16(o[:, :, torch.from_numpy(rows).cuda()])
         _check(out, oracle.attention(q, k, v, rows=rows), mode, case.name)
         assert torch.isfinite(o.float()).all().item()
+
+
+def test_video_long_workload_sampled_rows():
+    # The benchmark's workload (N=119056, K offsets) in the benchmark's launch:
+    # K-mean smoothing, FP8 PV; 64 sampled rows per head against all keys.
+    import diffusion_transformer_attention_attn_b200 as dit
+    case = inputs.VIDEO_LONG
+    q, k, v = inputs.attn_inputs(case)
+    o = dit.dit_attn_fwd_q8(*_dev(q, k, v), smooth_k=True, pv_mode="fp8")
+    torch.cuda.synchronize()
+    rows = inputs.sample_rows(case.N, 64)
+    out = from_device_bf16(o[:, :, torch.from_numpy(rows).cuda()])
+    _check(out, oracle.attention(q, k, v, rows=rows), "fp8", case.name)
+    assert torch.isfinite(o.float()).all().item()
