@@ -3,9 +3,13 @@
  * library (libditattn.so).
  *
  * The library holds the hot path of image and video diffusion transformers:
- * full bidirectional multi-head self-attention over one joint token stream,
- * and the first-block-cache residual difference that decides whether a
- * denoising step may reuse its cached residual.
+ * full bidirectional multi-head self-attention over one joint token stream
+ * (bf16, and 8-bit with INT8 QKᵀ and FP8 or bf16 PV), and the first-block-cache
+ * residual difference that decides whether a denoising step may reuse its
+ * cached residual.  Around them: attention over a chunk of the keys with its
+ * log-sum-exp and the merge of chunks, the 8-bit pre-pass split for a
+ * token-sharded sequence, the error of one output against another, and (in
+ * dit_cache.h) step-cache policies whose decisions stay on the device.
  *
  * Conventions shared by every entry point
  *   - Every buffer is caller-owned device memory.  The library allocates no
