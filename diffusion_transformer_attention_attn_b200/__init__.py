@@ -22,6 +22,10 @@ Entry points (same names as the C ABI in ``include/dit_attn.h``):
 and of ``include/dit_cache.h``:
   * ``fbcache_step(...)`` / ``teacache_step(...)``  — step-cache decisions kept on the device
   * ``dit_cache_state_reset``, ``dit_graph_*``     — device state and CUDA-graph conditional plumbing
+
+Modules on top: ``step_cache`` (a captured denoising step that skips its
+expensive part on cached steps) and ``context_parallel`` (Ulysses and ring
+attention, the sharded cache decision, over ``torch.distributed``).
 """
 from __future__ import annotations
 
