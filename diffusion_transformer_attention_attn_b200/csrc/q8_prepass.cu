@@ -74,17 +74,35 @@ __global__ void __launch_bounds__(kStatThreads)
         acc[i] = 0.0;
         vmax[i] = 0.f;
     }
-    for (int64_t n = n0 + r0; n < n1; n += kStatThreads / 16) {
-        float f[8];
-        if (want_sum) {
-            unpack8(__ldg(row_ptr(k, sb, sh, sn, b, h, n) + cg), f);
+    // Rows are visited in the same order as one at a time, but the loads of
+    // kBatch rows are issued before any of them is used.
+    constexpr int kStep = kStatThreads / 16;  // rows between a thread's rows
+    constexpr int kBatch = 4;
+    for (int64_t nb = n0 + r0; nb < n1; nb += kBatch * kStep) {
+        uint4 kr[kBatch], vr[kBatch];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] += static_cast<double>(f[i]);
+        for (int u = 0; u < kBatch; ++u) {
+            const int64_t n = nb + u * kStep;
+            if (n < n1) {
+                if (want_sum) kr[u] = __ldg(row_ptr(k, sb, sh, sn, b, h, n) + cg);
+                if (want_vmax) vr[u] = __ldg(row_ptr(v, sb, sh, sn, b, h, n) + cg);
+            }
         }
-        if (want_vmax) {
-            unpack8(__ldg(row_ptr(v, sb, sh, sn, b, h, n) + cg), f);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) vmax[i] = fmaxf(vmax[i], fabsf(f[i]));
+        for (int u = 0; u < kBatch; ++u) {
+            if (nb + u * kStep < n1) {
+                float f[8];
+                if (want_sum) {
+                    unpack8(kr[u], f);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] += static_cast<double>(f[i]);
+                }
+                if (want_vmax) {
+                    unpack8(vr[u], f);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) vmax[i] = fmaxf(vmax[i], fabsf(f[i]));
+                }
+            }
         }
     }
 #pragma unroll
@@ -107,19 +125,49 @@ __global__ void __launch_bounds__(kStatThreads)
     }
 }
 
-// grid B*H, 128 threads (one per channel).
-__global__ void q8_finalize_kernel(const double* __restrict__ psum, const float* __restrict__ pmax, int n_chunks,
-                                   int N, int want_sum, int want_vmax, float* __restrict__ k_mean,
-                                   float* __restrict__ v_scale, float* __restrict__ v_inv) {
+// Per (b,h) and channel: the partials' K sum and V maximum over all chunks.
+// kFinGroups × 128 threads; group g takes chunks g, g + kFinGroups, ... in
+// order, then thread (0, c) adds the groups' sums in group order, so the
+// result does not depend on timing.  Only group 0's (sum, max) are complete.
+constexpr int kFinGroups = 8;
+__device__ __forceinline__ void chunk_reduce(const double* __restrict__ psum, const float* __restrict__ pmax,
+                                             int n_chunks, int want_sum, int want_vmax, double& s_out,
+                                             float& m_out) {
     constexpr int D = 128;
-    const int bh = blockIdx.x, c = threadIdx.x;
+    __shared__ double s_part[kFinGroups][D];
+    __shared__ float m_part[kFinGroups][D];
+    const int bh = blockIdx.x, c = threadIdx.x & (D - 1), g = threadIdx.x / D;
     double s = 0.0;
     float m = 0.f;
-    for (int i = 0; i < n_chunks; ++i) {
+    for (int i = g; i < n_chunks; i += kFinGroups) {
         const int64_t idx = (static_cast<int64_t>(bh) * n_chunks + i) * D + c;
         if (want_sum) s += psum[idx];
         if (want_vmax) m = fmaxf(m, pmax[idx]);
     }
+    s_part[g][c] = s;
+    m_part[g][c] = m;
+    __syncthreads();
+    if (g == 0) {
+        for (int j = 1; j < kFinGroups; ++j) {
+            s += s_part[j][c];
+            m = fmaxf(m, m_part[j][c]);
+        }
+    }
+    s_out = s;
+    m_out = m;
+}
+
+// grid B*H, kFinGroups × 128 threads.
+__global__ void __launch_bounds__(kFinGroups * 128)
+    q8_finalize_kernel(const double* __restrict__ psum, const float* __restrict__ pmax, int n_chunks, int N,
+                       int want_sum, int want_vmax, float* __restrict__ k_mean, float* __restrict__ v_scale,
+                       float* __restrict__ v_inv) {
+    constexpr int D = 128;
+    const int bh = blockIdx.x, c = threadIdx.x;
+    double s;
+    float m;
+    chunk_reduce(psum, pmax, n_chunks, want_sum, want_vmax, s, m);
+    if (threadIdx.x >= D) return;
     k_mean[bh * D + c] = want_sum ? static_cast<float>(s / static_cast<double>(N)) : 0.f;
     if (want_vmax) {
         float sc = 0.f, inv = 0.f;
@@ -132,14 +180,19 @@ __global__ void q8_finalize_kernel(const double* __restrict__ psum, const float*
     }
 }
 
+// Four fp32 -> four int8 codes (round half to even, saturated to ±127);
+// element 0 in bits 0-7.  Clamping first and then adding 1.5·2^23 leaves the
+// rounded integer in the low mantissa bits of the sum (the add rounds to
+// nearest even), and its low byte is the two's-complement code.  The
+// quantisers' inputs are within one rounding of ±127, so this is the same
+// code as rounding first and saturating to the int8 range.
+__device__ __forceinline__ uint32_t s8_bits(float x) {
+    return __float_as_uint(__fadd_rn(fminf(fmaxf(x, -127.f), 127.f), 12582912.f));
+}
 __device__ __forceinline__ uint32_t s8x4(float a, float b, float c, float d) {
-    int ia, ib, ic, id;
-    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(ia) : "f"(a));
-    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(ib) : "f"(b));
-    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(ic) : "f"(c));
-    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(id) : "f"(d));
-    return (static_cast<uint32_t>(ia) & 0xFFu) | ((static_cast<uint32_t>(ib) & 0xFFu) << 8) |
-           ((static_cast<uint32_t>(ic) & 0xFFu) << 16) | ((static_cast<uint32_t>(id) & 0xFFu) << 24);
+    const uint32_t lo = __byte_perm(s8_bits(a), s8_bits(b), 0x0040);
+    const uint32_t hi = __byte_perm(s8_bits(c), s8_bits(d), 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
 }
 
 // INT8 per block of BLK tokens.  grid (ceil(N/BLK), B*H), 256 threads:
@@ -235,19 +288,16 @@ __global__ void __launch_bounds__(kQuantThreads)
 
 // Token-sharded form (one slice of the tokens per device): the per-channel
 // K sums and V maxima of this slice, for the devices to combine.  grid B*H,
-// 128 threads (one per channel); the same fixed-order sum as q8_finalize.
-__global__ void q8_slice_stats_kernel(const double* __restrict__ psum, const float* __restrict__ pmax, int n_chunks,
-                                      int want_sum, int want_vmax, double* __restrict__ k_sum,
-                                      float* __restrict__ v_amax) {
+// kFinGroups × 128 threads; the same fixed-order sum as q8_finalize.
+__global__ void __launch_bounds__(kFinGroups * 128)
+    q8_slice_stats_kernel(const double* __restrict__ psum, const float* __restrict__ pmax, int n_chunks,
+                          int want_sum, int want_vmax, double* __restrict__ k_sum, float* __restrict__ v_amax) {
     constexpr int D = 128;
     const int bh = blockIdx.x, c = threadIdx.x;
-    double s = 0.0;
-    float m = 0.f;
-    for (int i = 0; i < n_chunks; ++i) {
-        const int64_t idx = (static_cast<int64_t>(bh) * n_chunks + i) * D + c;
-        if (want_sum) s += psum[idx];
-        if (want_vmax) m = fmaxf(m, pmax[idx]);
-    }
+    double s;
+    float m;
+    chunk_reduce(psum, pmax, n_chunks, want_sum, want_vmax, s, m);
+    if (threadIdx.x >= D) return;
     k_sum[bh * D + c] = s;
     v_amax[bh * D + c] = m;
 }
@@ -307,7 +357,7 @@ cudaError_t launch_q8_prepass(const void* q, const void* k, const void* v, int64
     if (smooth_k || pv_fp8) {
         q8_stats_kernel<<<dim3(L.n_chunks, BH), kStatThreads, 0, stream>>>(k, v, sb, sh, sn, H, N, kQ8StatChunk,
                                                                            smooth_k, pv_fp8, psum, pmax);
-        q8_finalize_kernel<<<BH, 128, 0, stream>>>(psum, pmax, L.n_chunks, N, smooth_k, pv_fp8, k_mean, v_scale,
+        q8_finalize_kernel<<<BH, kFinGroups * 128, 0, stream>>>(psum, pmax, L.n_chunks, N, smooth_k, pv_fp8, k_mean, v_scale,
                                                    v_inv);
     }
     return launch_q8_codes(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, stream);
@@ -341,7 +391,7 @@ cudaError_t launch_q8_slice_stats(const void* k, const void* v, int64_t sb, int6
     if (smooth_k || pv_fp8)
         q8_stats_kernel<<<dim3(L.n_chunks, BH), kStatThreads, 0, stream>>>(k, v, sb, sh, sn, H, N, kQ8StatChunk,
                                                                            smooth_k, pv_fp8, psum, pmax);
-    q8_slice_stats_kernel<<<BH, 128, 0, stream>>>(psum, pmax, L.n_chunks, smooth_k, pv_fp8, k_sum, v_amax);
+    q8_slice_stats_kernel<<<BH, kFinGroups * 128, 0, stream>>>(psum, pmax, L.n_chunks, smooth_k, pv_fp8, k_sum, v_amax);
     return cudaGetLastError();
 }
 
