@@ -19,7 +19,7 @@
 // faster.)
 // Tensor memory (512 columns × 128 lanes × 32 bit):
 //   [0,128)  S0 = Q0·Kᵀ (fp32); after the softmax, P0 (bf16 pairs) in [0,64),
-//            written and published in two 64-key halves
+//            written in two 64-key halves and published once whole (kSplitP)
 //   [128,256) S1 / P1
 //   [256,256+d) O0 accumulator;  [256+d, 256+2d) O1 accumulator
 // The MMA warp alternates the two tiles so that the tensor core computes
@@ -384,9 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // P = 2^(s·scale·log2e − m): packed FFMA, ex2 (MUFU, or the FMA
             // pipe for kEmuOf8 pairs in 8), packed row sum, bf16 pairs into
-            // tensor memory.  Each 64-key half is published as soon as it is
-            // written, so its P·V MMAs start while the next half is computed.
-            // Keys past N get P = 0.
+            // tensor memory, one 64-key half at a time.  With kSplitP each half
+            // is published as soon as it is written (its P·V MMAs then start
+            // while the next half is computed); otherwise P is published once
+            // whole.  Keys past N get P = 0.
             const float2 c2 = make_float2(scale_log2, scale_log2);
             const float2 negm2 = make_float2(-m, -m);
             float2 ls[4];
