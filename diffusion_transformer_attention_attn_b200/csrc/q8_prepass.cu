@@ -180,30 +180,28 @@ __global__ void __launch_bounds__(kFinGroups * 128)
     }
 }
 
-// Four fp32 -> four int8 codes (round half to even, saturated to ±127);
-// element 0 in bits 0-7.  Clamping first and then adding 1.5·2^23 leaves the
-// rounded integer in the low mantissa bits of the sum (the add rounds to
-// nearest even), and its low byte is the two's-complement code.  The
-// quantisers' inputs are within one rounding of ±127, so this is the same
-// code as rounding first and saturating to the int8 range.
-__device__ __forceinline__ uint32_t s8_bits(float x) {
-    return __float_as_uint(__fadd_rn(fminf(fmaxf(x, -127.f), 127.f), 12582912.f));
-}
 __device__ __forceinline__ uint32_t s8x4(float a, float b, float c, float d) {
-    const uint32_t lo = __byte_perm(s8_bits(a), s8_bits(b), 0x0040);
-    const uint32_t hi = __byte_perm(s8_bits(c), s8_bits(d), 0x0040);
-    return __byte_perm(lo, hi, 0x5410);
+    int ia, ib, ic, id;
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(ia) : "f"(a));
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(ib) : "f"(b));
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(ic) : "f"(c));
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(id) : "f"(d));
+    return (static_cast<uint32_t>(ia) & 0xFFu) | ((static_cast<uint32_t>(ib) & 0xFFu) << 8) |
+           ((static_cast<uint32_t>(ic) & 0xFFu) << 16) | ((static_cast<uint32_t>(id) & 0xFFu) << 24);
 }
 
-// INT8 per block of BLK tokens.  grid (ceil(N/BLK), B*H), 256 threads:
-// thread t holds channels [8·(t%16), +8) of rows t/16 + 16·i of the block.
-template <int BLK>
-__global__ void __launch_bounds__(kQuantThreads)
+// INT8 per block of BLK tokens.  grid (ceil(N/BLK), B*H), THREADS threads:
+// thread t holds channels [8·(t%16), +8) of rows t/16 + (THREADS/16)·i of
+// the block (Q: 128 tokens on 512 threads, K: 64 tokens on 256 threads).
+// Codes are cvt.rni.sat.s8.f32 of x·inv: round half to even, saturated.
+template <int BLK, int THREADS>
+__global__ void __launch_bounds__(THREADS)
     q8_quant_int8_kernel(const void* __restrict__ x, int64_t sb, int64_t sh, int64_t sn, int H, int N,
                          const float* __restrict__ mean, int8_t* __restrict__ codes, float* __restrict__ scales) {
     constexpr int D = 128;
-    constexpr int kRows = BLK / 16;  // rows per thread
-    __shared__ float s_red[kQuantThreads / 32];
+    constexpr int kGroups = THREADS / 16;  // row groups
+    constexpr int kRows = BLK / kGroups;   // rows per thread
+    __shared__ float s_red[THREADS / 32];
     const int bh = blockIdx.y, b = bh / H, h = bh % H;
     const int cg = threadIdx.x & 15, r0 = threadIdx.x >> 4;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * BLK;
@@ -214,7 +212,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     float amax = 0.f;
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
-        const int64_t n = t0 + r0 + 16 * r;
+        const int64_t n = t0 + r0 + kGroups * r;
         if (n < N) {
             unpack8(__ldg(row_ptr(x, sb, sh, sn, b, h, n) + cg), val[r]);
 #pragma unroll
@@ -230,7 +228,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     __syncthreads();
     amax = s_red[0];
 #pragma unroll
-    for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, s_red[w]);
+    for (int w = 1; w < THREADS / 32; ++w) amax = fmaxf(amax, s_red[w]);
     float inv = 0.f, scale = 0.f;
     if (amax > 0.f) {  // zero-scale guard
         inv = __fdiv_rn(127.f, amax);
@@ -239,7 +237,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     if (threadIdx.x == 0) scales[static_cast<int64_t>(bh) * gridDim.x + blockIdx.x] = scale;
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
-        const int64_t n = t0 + r0 + 16 * r;
+        const int64_t n = t0 + r0 + kGroups * r;
         if (n < N) {
             float q[8];
 #pragma unroll
@@ -369,10 +367,10 @@ cudaError_t launch_q8_codes(const void* q, const void* k, const void* v, int64_t
     const int BH = B * H;
     const float* k_mean = reinterpret_cast<const float*>(ws + L.k_mean);
     const float* v_inv = reinterpret_cast<const float*>(ws + L.v_inv);
-    q8_quant_int8_kernel<128><<<dim3((N + 127) / 128, BH), kQuantThreads, 0, stream>>>(
+    q8_quant_int8_kernel<128, 512><<<dim3((N + 127) / 128, BH), 512, 0, stream>>>(
         q, sb, sh, sn, H, N, nullptr, reinterpret_cast<int8_t*>(ws + L.q_codes),
         reinterpret_cast<float*>(ws + L.q_scale));
-    q8_quant_int8_kernel<64><<<dim3((N + 63) / 64, BH), kQuantThreads, 0, stream>>>(
+    q8_quant_int8_kernel<64, 256><<<dim3((N + 63) / 64, BH), 256, 0, stream>>>(
         k, sb, sh, sn, H, N, smooth_k ? k_mean : nullptr, reinterpret_cast<int8_t*>(ws + L.k_codes),
         reinterpret_cast<float*>(ws + L.k_scale));
     if (pv_fp8)
