@@ -18,6 +18,7 @@ Entry points (same names as the C ABI in ``include/dit_attn.h``):
   * ``fbc_rel_l1_noalloc(...)``                     — the same, allocating nothing
   * ``dit_compare_stats(ref, test, segments)``       — rel-L1 / cosine / max error per segment
   * ``dit_get_device_status()``                     — device-side error word
+  * ``dit_wait_selftest()``                         — makes a bounded wait run out (failure-path test)
 
 and of ``include/dit_cache.h``:
   * ``fbcache_step(...)`` / ``teacache_step(...)``  — step-cache decisions kept on the device
@@ -72,6 +73,7 @@ SIGNATURES = {
     "dit_compare_workspace_bytes": (_sz, [_i64, _i64, _i]),
     "dit_compare_stats": (_i, [_p, _p, _i64, _i64, _i, _p, _p, _sz, _p]),
     "dit_get_device_status": (_i, [_p]),
+    "dit_wait_selftest": (_i, [_p, _p]),
     "dit_status_string": (ctypes.c_char_p, [_i]),
     # include/dit_cache.h
     "dit_cache_state_reset": (_i, [_p, _p]),
@@ -500,6 +502,19 @@ def fbc_rel_l1_noalloc(r_cur, r_prev, threshold: float, out_rel, out_skip, strea
 def dit_get_device_status(stream=None) -> int:
     """Synchronise the stream; return (and clear) the device error word."""
     return int(load_library().dit_get_device_status(_stream_ptr(stream)))
+
+
+def dit_wait_selftest(stream=None) -> int:
+    """Run the bounded-wait self-test (about 1 s on the stream).  Returns the
+    kernel's 'completed' flag: 0 when the wait gave up, as it must.  The device
+    error word then holds DIT_ERR_TIMEOUT (read it with dit_get_device_status)."""
+    import torch
+    lib = load_library()
+    s = torch.cuda.current_stream() if stream is None else stream
+    flag = torch.full((1,), -1, dtype=torch.int32, device=s.device)
+    _check(lib.dit_wait_selftest(flag.data_ptr(), _stream_ptr(stream)), "dit_wait_selftest")
+    s.synchronize()
+    return int(flag.item())
 
 
 def dit_compare_workspace_bytes(n_segments: int, segment_len: int, dtype) -> int:

@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libditattn.so")
 
 SOURCES = ["api.cu", "attn_bf16.cu", "attn_bf16_ks.cu", "attn_q8.cu", "q8_prepass.cu", "attn_merge.cu", "fbc_rel_l1.cu", "cache_step.cu",
-           "compare.cu"]
+           "compare.cu", "selftest.cu"]
 HEADERS = ["sm100_ptx.cuh", "internal.h", "rel_l1_reduce.cuh"]
 
 NVCC_FLAGS = [

@@ -2,7 +2,8 @@
 // validation, TMA tensor-map encoding and launches.  Host code only; the
 // arithmetic of every call runs in the kernels of attn_bf16.cu, attn_q8.cu,
 // q8_prepass.cu, attn_merge.cu and fbc_rel_l1.cu (the step caches and the output comparison
-// have their own entry points in cache_step.cu and compare.cu).
+// have their own entry points in cache_step.cu and compare.cu; the bounded-wait self-test
+// kernel is in selftest.cu).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -481,6 +482,15 @@ dit_status fbc_rel_l1_finish(const double* sums, float threshold, double* out_re
     dit_status st;
     if (!device_state(&st)) return st;
     cudaError_t e = launch_fbc_finish(sums, threshold, out_rel, out_skip, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+dit_status dit_wait_selftest(int32_t* out_completed, void* stream) {
+    if (out_completed == nullptr) return DIT_ERR_INVALID_ARG;
+    dit_status st;
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    const cudaError_t e = launch_wait_selftest(ds->err_word, out_completed, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 

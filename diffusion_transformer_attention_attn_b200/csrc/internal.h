@@ -24,6 +24,11 @@ cudaError_t launch_attn_bf16_ks(const CUtensorMap& tq, const CUtensorMap& tk, co
                                 int64_t sb, int64_t sh, int64_t sn, int B, int H, int Nq, int Nkv, int d,
                                 float scale_log2, float* lse, int* err, cudaStream_t stream);
 
+// Bounded-wait self-test (selftest.cu): one warp waits on an mbarrier that is
+// never arrived on, gives up after the wait limit and records DIT_ERR_TIMEOUT
+// in *err; *completed gets 0 (1 would mean the wait ended normally).
+cudaError_t launch_wait_selftest(int* err, int32_t* completed, cudaStream_t stream);
+
 // Merge of per-key-chunk outputs (see dit_attn_merge in dit_attn.h).
 constexpr int kMaxMergeParts = 16;
 cudaError_t launch_attn_merge(const void* const* o_parts, const float* const* lse_parts, int n_parts, int B, int H,

@@ -320,6 +320,21 @@ dit_status dit_compare_stats(const void* ref, const void* test, int64_t n_segmen
  */
 dit_status dit_get_device_status(void* stream);
 
+/*
+ * dit_wait_selftest — exercises the bounded wait that every kernel of this
+ * library uses (no page counterpart: it tests the library's own failure
+ * detection).  One warp waits on an mbarrier that nothing arrives on, gives
+ * up after the wait limit (1 s), records DIT_ERR_TIMEOUT in the device error
+ * word and returns, leaving the GPU context usable.
+ *   out_completed  device int32 [1]; set to 0 when the wait gave up (1 would
+ *                  mean the barrier completed, which cannot happen).
+ * Asynchronous on `stream` (it occupies the stream for about 1 s); read the
+ * outcome with dit_get_device_status, which then returns DIT_ERR_TIMEOUT.
+ * Returns DIT_ERR_INVALID_ARG for a NULL out_completed, DIT_ERR_CUDA if the
+ * launch fails.
+ */
+dit_status dit_wait_selftest(int32_t* out_completed, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* dit_status_string(int status);
 

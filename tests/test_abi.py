@@ -308,3 +308,7 @@ def test_sharded_q8_argument_errors(lib):
     assert pq(scale=float("nan")) == dit.DIT_ERR_INVALID_ARG
     assert pq(wsb=1) == dit.DIT_ERR_WORKSPACE
     assert pq(ws=WS + 128) == dit.DIT_ERR_WORKSPACE
+
+
+def test_wait_selftest_argument_error(lib):
+    assert lib.dit_wait_selftest(None, None) == dit.DIT_ERR_INVALID_ARG
