@@ -12,7 +12,7 @@ zero-scale guard (TMAP page, "optimising operator details").
 
 ``emulated_q8_attention`` is parity unpinned beyond its inputs: it replays the
 quantised arithmetic in fp64 to separate quantisation error from kernel error
-and is never the judged reference (the judged reference for the 8-bit path is
+and is never the parity reference (the parity reference for the 8-bit path is
 the exact fp64 attention on the unquantised inputs).
 """
 from __future__ import annotations

@@ -129,7 +129,7 @@ def test_batch_heads_and_explicit_scale(mode):
 
 @pytest.mark.parametrize("mode", ["bf16", "fp8"])
 def test_image_q8_workload_sampled_rows(mode):
-    # The 8-bit image workload at full size (N=4608), smooth_k on (judged).
+    # The 8-bit image workload at full size (N=4608), smooth_k on (held to the 8-bit tolerances).
     import diffusion_transformer_attention_attn_b200 as dit
     case = inputs.IMAGE_Q8
     q, k, v = inputs.attn_inputs(case)
@@ -143,7 +143,7 @@ def test_image_q8_workload_sampled_rows(mode):
 
 def test_image_q8_without_smoothing_reported():
     # smooth_k = 0: K's per-channel offsets (std 5) set the INT8 scale, so the
-    # N(0,1) part is quantised coarsely.  Reported, not judged: finite, and
+    # N(0,1) part is quantised coarsely.  Reported, not held to the tolerances: finite, and
     # still strongly correlated with the exact result.
     import diffusion_transformer_attention_attn_b200 as dit
     case = inputs.IMAGE_Q8
