@@ -195,7 +195,7 @@ __device__ __forceinline__ uint32_t s8x4(float a, float b, float c, float d) {
 // the block (Q: 128 tokens on 512 threads, K: 64 tokens on 256 threads).
 // Codes are cvt.rni.sat.s8.f32 of x·inv: round half to even, saturated.
 template <int BLK, int THREADS>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, 1536 / THREADS)
     q8_quant_int8_kernel(const void* __restrict__ x, int64_t sb, int64_t sh, int64_t sn, int H, int N,
                          const float* __restrict__ mean, int8_t* __restrict__ codes, float* __restrict__ scales) {
     constexpr int D = 128;
@@ -208,18 +208,24 @@ __global__ void __launch_bounds__(THREADS)
     float mu[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) mu[i] = mean ? mean[bh * D + cg * 8 + i] : 0.f;
-    float val[kRows][8];
+    // The rows stay in registers as loaded (bf16), and are widened again for
+    // the codes: half the registers of keeping fp32 values, so more blocks
+    // fit on an SM and more loads are in flight.
+    uint4 raw[kRows];
     float amax = 0.f;
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
         const int64_t n = t0 + r0 + kGroups * r;
-        if (n < N) {
-            unpack8(__ldg(row_ptr(x, sb, sh, sn, b, h, n) + cg), val[r]);
+        if (n < N) raw[r] = __ldg(row_ptr(x, sb, sh, sn, b, h, n) + cg);
+    }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (mean) val[r][i] = __fsub_rn(val[r][i], mu[i]);
-                amax = fmaxf(amax, fabsf(val[r][i]));
-            }
+    for (int r = 0; r < kRows; ++r) {
+        const int64_t n = t0 + r0 + kGroups * r;
+        if (n < N) {
+            float f[8];
+            unpack8(raw[r], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(mean ? __fsub_rn(f[i], mu[i]) : f[i]));
         }
     }
 #pragma unroll
@@ -239,9 +245,10 @@ __global__ void __launch_bounds__(THREADS)
     for (int r = 0; r < kRows; ++r) {
         const int64_t n = t0 + r0 + kGroups * r;
         if (n < N) {
-            float q[8];
+            float f[8], q[8];
+            unpack8(raw[r], f);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(val[r][i], inv);
+            for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(mean ? __fsub_rn(f[i], mu[i]) : f[i], inv);
             uint2 w;
             w.x = s8x4(q[0], q[1], q[2], q[3]);
             w.y = s8x4(q[4], q[5], q[6], q[7]);
