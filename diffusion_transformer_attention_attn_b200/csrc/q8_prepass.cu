@@ -56,7 +56,9 @@ __device__ __forceinline__ const uint4* row_ptr(const void* base, int64_t sb, in
 }
 
 // grid (n_chunks, B*H).  Thread t: 8 channels [8·(t%16), +8), rows t/16 + 16·i.
-__global__ void __launch_bounds__(kStatThreads)
+// Four blocks per SM (64 registers) keep more loads in flight than two
+// blocks with deeper per-thread batches.
+__global__ void __launch_bounds__(kStatThreads, 4)
     q8_stats_kernel(const void* __restrict__ k, const void* __restrict__ v, int64_t sb, int64_t sh, int64_t sn, int H,
                     int N, int chunk, int want_sum, int want_vmax, double* __restrict__ psum,
                     float* __restrict__ pmax) {
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(kStatThreads)
     // Rows are visited in the same order as one at a time, but the loads of
     // kBatch rows are issued before any of them is used.
     constexpr int kStep = kStatThreads / 16;  // rows between a thread's rows
-    constexpr int kBatch = 4;
+    constexpr int kBatch = 2;
     for (int64_t nb = n0 + r0; nb < n1; nb += kBatch * kStep) {
         uint4 kr[kBatch], vr[kBatch];
 #pragma unroll
