@@ -19,7 +19,7 @@
 // faster.)
 // Tensor memory (512 columns × 128 lanes × 32 bit):
 //   [0,128)  S0 = Q0·Kᵀ (fp32); after the softmax, P0 (bf16 pairs) in [0,64),
-//            written in two 64-key halves and published once whole (kSplitP)
+//            written and published in two 64-key halves (kSplitP)
 //   [128,256) S1 / P1
 //   [256,256+d) O0 accumulator;  [256+d, 256+2d) O1 accumulator
 // The MMA warp alternates the two tiles so that the tensor core computes
@@ -62,8 +62,8 @@ constexpr int kOtherRegs = 72;
 // Pairs of exponentials (out of every 8) evaluated on the FMA pipe.
 constexpr int kEmuOf8 = 1;
 // Publish P in two 64-key halves (the MMA warp starts P·V on the first half
-// while the second is computed) or whole.
-constexpr bool kSplitP = false;
+// while the second is computed) or whole.  Halves measured 2% faster.
+constexpr bool kSplitP = true;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
