@@ -10,10 +10,12 @@ image-to-video page, FLOP table), the first-block-cache residual difference
 (ParaAttention page, "First Block Cache") and the 8-bit quantiser with its
 zero-scale guard (TMAP page, "optimising operator details").
 
-``emulated_q8_attention`` is parity unpinned beyond its inputs: it replays the
-quantised arithmetic in fp64 to separate quantisation error from kernel error
-and is never the parity reference (the parity reference for the 8-bit path is
-the exact fp64 attention on the unquantised inputs).
+``emulated_q8_attention`` and ``attention_from_codes`` replay the quantised
+arithmetic in fp64 to separate quantisation error from kernel error; they are
+never the parity reference (that is the exact fp64 attention on the
+unquantised inputs).  They are pinned on inputs whose every code is exact, with
+a different scale in each Q and K block, where they must equal the exact
+attention.
 """
 from __future__ import annotations
 
@@ -177,7 +179,7 @@ def e4m3_decode(b: np.ndarray) -> np.ndarray:
 
 def emulated_q8_attention(q, k, v, scale: float | None = None, smooth_k: bool = True,
                           rows=None) -> np.ndarray:
-    """fp64 attention over the dequantised 8-bit inputs (parity unpinned).
+    """fp64 attention over the dequantised 8-bit inputs.
 
     Replays the quantiser (Q per 128 tokens, K per 64 tokens after the optional
     channel-mean subtraction, V per channel e4m3) and runs the exact fp64
@@ -327,12 +329,15 @@ def mean_from_sums(sums: np.ndarray, n_total: int) -> np.ndarray:
 def quant_e4m3_with_amax(x: np.ndarray, amax: np.ndarray):
     """Per-channel e4m3 codes of x [B,H,N,d] (bf16 bits) with the channel maxima
     given ([B,H,d] fp32): scale = amax/448 and inv = 448/amax as fp32
-    divisions, code = e4m3(x·inv) (fp32 product); amax = 0 gives zero codes
-    and scales (the zero-scale guard).  Returns (codes, scales)."""
+    divisions, code = e4m3(x·inv) (fp32 product); amax = 0, or an amax whose
+    inverse 448/amax is not a finite fp32 number, gives zero codes and scales
+    (the zero-scale guard).  Returns (codes, scales)."""
     amax = np.asarray(amax, dtype=np.float32)
-    with np.errstate(divide="ignore"):
-        scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(0.0)).astype(np.float32)
-        inv = np.where(amax > 0, np.float32(448.0) / amax, np.float32(0.0)).astype(np.float32)
+    with np.errstate(divide="ignore", over="ignore"):
+        inv_raw = (np.float32(448.0) / amax).astype(np.float32)
+        ok = (amax > 0) & np.isfinite(inv_raw)
+        scale = np.where(ok, amax / np.float32(448.0), np.float32(0.0)).astype(np.float32)
+        inv = np.where(ok, inv_raw, np.float32(0.0)).astype(np.float32)
     xf = _widen(x).astype(np.float32)
     prod = (xf * inv[:, :, None, :]).astype(np.float32)
     return e4m3_encode(prod), scale

@@ -38,10 +38,12 @@
  *    quantisation ("128*128 per-block quantisation operator" in the same
  *    section).  Readings: amax over the valid tokens of a block and all its
  *    channels; inv = 127/amax and scale = amax/127 as fp32 divisions;
- *    code = round-half-even(x*inv) clamped to [-127, 127]; amax == 0 gives
+ *    code = round-half-even(x*inv) clamped to [-127, 127]; amax == 0, or an
+ *    amax so small that 127/amax is not a finite fp32 number, gives
  *    scale = inv = 0 and all-zero codes.  The K mean is summed in fp64 and
  *    rounded to fp32, then subtracted in fp32.  V: per-channel amax over the
- *    valid tokens, scale = amax/448, inv = 448/amax, the same zero guard.
+ *    valid tokens, scale = amax/448, inv = 448/amax, the same zero guard
+ *    (amax zero, or 448/amax not finite).
  *
  *  - An FP8 E4M3 encoder written from the OCP 8-bit floating point
  *    specification (bias 7, 3 mantissa bits, no infinities, 0x7F/0xFF NaN,
@@ -314,7 +316,11 @@ int oracle_quant_int8_blocks(const uint16_t *x, int64_t BH, int64_t N, int64_t d
                         amax = a;
                 }
             float inv = 0.0f, scale = 0.0f;
-            if (amax > 0.0f) { /* zero-scale guard */
+            /* zero-scale guard: an amax of zero, or one so small that
+             * 127/amax overflows fp32 (below about 3.7e-37), makes the block
+             * all-zero codes with scale 0; an infinite inv would turn the
+             * block's exact zeros into 0 * inf = NaN. */
+            if (amax > 0.0f && isfinite(127.0f / amax)) {
                 inv = 127.0f / amax;
                 scale = amax / 127.0f;
             }
@@ -391,7 +397,9 @@ int oracle_quant_e4m3_channels(const uint16_t *x, int64_t BH, int64_t N, int64_t
                     amax = a;
             }
             float inv = 0.0f, scale = 0.0f;
-            if (amax > 0.0f) {
+            /* the same guard: amax zero, or 448/amax not finite (amax below
+             * about 1.3e-36), gives zero codes and scale 0 */
+            if (amax > 0.0f && isfinite(448.0f / amax)) {
                 inv = 448.0f / amax;
                 scale = amax / 448.0f;
             }

@@ -381,3 +381,96 @@ def test_fbc_sums_of_shards_add_up_and_give_rel():
     assert oracle.fbc_sums(np.float32([1.5, -2, 2, -4]), np.float32([1, -2, 3, -4])) == (1.5, 10.0)
     assert oracle.rel_from_sums(0.0, 0.0, 0.1) == (0.0, 1)
     assert oracle.rel_from_sums(1.0, 0.0, 0.1) == (float("inf"), 0)
+
+
+# ---------------------------------------------------------------- 8-bit block-scale indexing
+
+def _scaled_blocks(rng, n_tok, d, blk, halves):
+    """Values exactly representable after INT8 quantisation: block b holds
+    integers in [-127, 127] with 127 present (amax 127: inv 1, scale 1) when
+    halves[b] is False, else multiples of 1/2 in [-63.5, 63.5] with 63.5
+    present (amax 63.5: inv 2, scale 1/2).  The second half of each block is
+    the negation of its first half, so every channel's mean is exactly 0."""
+    x = np.empty((1, 1, n_tok, d), dtype=np.float32)
+    for b in range(n_tok // blk):
+        half = rng.integers(-127, 128, (blk // 2, d)).astype(np.float32)
+        half[0, 0] = 127.0
+        if halves[b]:
+            half = half / np.float32(2.0)
+        x[0, 0, b * blk:b * blk + blk // 2] = half
+        x[0, 0, b * blk + blk // 2:(b + 1) * blk] = -half
+    return x
+
+
+@pytest.mark.parametrize("smooth_k", [False, True])
+def test_q8_dequantisation_uses_each_tokens_own_block_scale(smooth_k):
+    # Q blocks of 128 tokens with scales 1, 1/2; K blocks of 64 tokens with
+    # scales 1, 1/2, 1, 1/2; V e4m3-representable with channel maxima 448.
+    # Every code is exact, so both quantised-attention replays equal the exact
+    # attention; a swapped (64 <-> 128) or shifted block index does not.
+    rng = np.random.Generator(np.random.PCG64(77))
+    N, d, s = 256, 8, 1e-4
+    q = _scaled_blocks(rng, N, d, 128, [False, True])
+    k = _scaled_blocks(rng, N, d, 64, [False, True, False, True])
+    reps = oracle.e4m3_decode(np.arange(0, 127, dtype=np.uint8))
+    v = rng.choice(reps, (1, 1, N, d)).astype(np.float32) * rng.choice([-1.0, 1.0], (1, 1, N, d)).astype(np.float32)
+    v[0, 0, 5, :] = 448.0
+    qb, kb, vb = (inputs.bf16_bits(t) for t in (q, k, v))
+    exact = oracle.attention(qb, kb, vb, scale=s)
+    qc, qs = oracle.quant_int8_blocks(qb, 128)
+    kc, ks = oracle.quant_int8_blocks(kb, 64, oracle.channel_mean(kb) if smooth_k else None)
+    vc, vs = oracle.quant_e4m3_channels(vb)
+    np.testing.assert_array_equal(qs[0, 0], [1.0, 0.5])
+    np.testing.assert_array_equal(ks[0, 0], [1.0, 0.5, 1.0, 0.5])
+    np.testing.assert_array_equal(vs, np.ones((1, 1, d), dtype=np.float32))
+    emu = oracle.emulated_q8_attention(qb, kb, vb, scale=s, smooth_k=smooth_k)
+    np.testing.assert_allclose(emu, exact, rtol=0, atol=1e-12)
+    codes = oracle.attention_from_codes(qc, qs, kc, ks, vc, vs, scale=s)
+    np.testing.assert_allclose(codes, exact, rtol=0, atol=1e-12)
+    # The same replay with a wrong block index is far off: this input tells
+    # the indexings apart.
+    tok = np.arange(N)
+    vd = oracle.e4m3_decode(vc).astype(np.float64)
+    for qi, ki in ((np.minimum(tok // 64, 1), tok // 64),           # Q indexed per 64 tokens
+                   (tok // 128, np.minimum(tok // 128, 3)),         # K indexed per 128 tokens
+                   (tok // 128, (tok // 64 + 1) % 4)):              # K shifted by one block
+        wrong = oracle.attention(qc * qs[:, :, qi, None].astype(np.float64),
+                                 kc * ks[:, :, ki, None].astype(np.float64), vd, scale=s)
+        assert np.abs(wrong - exact).max() > 1e-2
+
+
+# ---------------------------------------------------------------- zero-scale guard, tiny maxima
+
+def test_zero_scale_guard_covers_maxima_without_a_finite_inverse():
+    # TMAP page, operator details: the quantisation scale of an all-zero
+    # channel made the output NaN.  The same happens when amax is so small
+    # that 127/amax (or 448/amax) overflows fp32: inv = inf and 0 * inf = NaN.
+    # Such a block or channel counts as zero; one whose inverse is finite is
+    # quantised normally.
+    x = np.zeros((1, 1, 384, 4), dtype=np.float32)
+    x[0, 0, 1:128:3, 2] = 1e-37                   # block 0: amax 1e-37, 127/amax overflows
+    x[0, 0, 128:256, :] = 1e-36                    # block 1: 127/1e-36 = 1.27e38, finite
+    x[0, 0, 130, 1] = 0.0
+    x[0, 0, 256:384, :] = 0.0                      # block 2: all zero
+    xb = inputs.bf16_bits(x)
+    codes, scales = oracle.quant_int8_blocks(xb, 128)
+    assert scales[0, 0, 0] == 0.0 and (codes[0, 0, :128] == 0).all()
+    a1 = np.float32(inputs.bf16_to_f32(xb)[0, 0, 128, 0])
+    assert scales[0, 0, 1] == a1 / np.float32(127) and scales[0, 0, 1] > 0
+    assert (codes[0, 0, 128:256][x[0, 0, 128:256] != 0] == 127).all() and codes[0, 0, 130, 1] == 0
+    assert scales[0, 0, 2] == 0.0 and (codes[0, 0, 256:] == 0).all()
+    # V per channel: channel 0 holds {0, 1e-37}, channel 1 has amax 1e-36
+    # (448/1e-36 overflows too), channel 2 amax 1e-35 (finite inverse).
+    v = np.zeros((1, 1, 64, 3), dtype=np.float32)
+    v[0, 0, ::2, 0] = 1e-37
+    v[0, 0, 3, 1] = 1e-36
+    v[0, 0, 7, 2] = 1e-35
+    vb = inputs.bf16_bits(v)
+    vc, vs = oracle.quant_e4m3_channels(vb)
+    assert vs[0, 0, 0] == 0.0 and vs[0, 0, 1] == 0.0 and vs[0, 0, 2] > 0
+    assert (vc[0, 0, :, :2] == 0).all() and vc[0, 0, 7, 2] == 0x7E    # 448 -> largest e4m3
+    amax = np.abs(inputs.bf16_to_f32(vb)).max(axis=2)
+    vc2, vs2 = oracle.quant_e4m3_with_amax(vb, amax)
+    np.testing.assert_array_equal(vc2, vc)
+    np.testing.assert_array_equal(vs2, vs)
+    assert np.isfinite(oracle.e4m3_decode(vc)).all()
