@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libditattn.so")
 
-SOURCES = ["api.cu", "attn_bf16.cu", "attn_bf16_ks.cu", "attn_q8.cu", "q8_prepass.cu", "attn_merge.cu", "fbc_rel_l1.cu", "cache_step.cu",
+SOURCES = ["api.cu", "attn_bf16.cu", "attn_q8.cu", "q8_prepass.cu", "attn_merge.cu", "fbc_rel_l1.cu", "cache_step.cu",
            "compare.cu", "selftest.cu"]
 HEADERS = ["sm100_ptx.cuh", "internal.h", "rel_l1_reduce.cuh"]
 
@@ -50,16 +50,12 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, key_split: bool = False) -> str:
-    """Compile the library.  key_split selects the key-split bf16 attention
-    schedule (attn_bf16_ks.cu) for dit_attn_fwd / dit_attn_fwd_ex instead of
-    the two-query-tile one (attn_bf16.cu)."""
-    if not force and not key_split and up_to_date():
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile the library (skipped when it is newer than every source)."""
+    if not force and up_to_date():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc_path(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC]
-    if key_split:
-        cmd += ["-DDIT_ATTN_KS"]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, s) for s in SOURCES]
@@ -73,10 +69,8 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true", help="pass -Xptxas -v (registers, spills, smem)")
-    ap.add_argument("--key-split", action="store_true",
-                    help="use the key-split bf16 attention schedule (one query tile per CTA)")
     a = ap.parse_args(argv)
-    print(build(force=a.force or a.verbose, verbose=a.verbose, key_split=a.key_split))
+    print(build(force=a.force or a.verbose, verbose=a.verbose))
 
 
 if __name__ == "__main__":

@@ -14,12 +14,6 @@
 #include "dit_attn.h"
 #include "internal.h"
 
-#ifdef DIT_ATTN_KS
-#define ATTN_BF16_LAUNCH launch_attn_bf16_ks
-#else
-#define ATTN_BF16_LAUNCH launch_attn_bf16
-#endif
-
 namespace ditk {
 
 // Device-side error word (one per device that loads the library); kernels
@@ -164,24 +158,27 @@ dit_status resolve_strides(const int64_t* strides, int B, int H, int N, int d, i
     return DIT_OK;
 }
 
-// 4-D map {128 B, N, H, B} over contiguous 8-bit codes [B, H, N, 128] inside
-// the workspace, box {128, 128, 1, 1}, 128-B swizzle.
-dit_status encode_u8_map(CUtensorMap* map, const void* base, int B, int H, int N) {
+// 4-D map {d B, N, H, B} over contiguous 8-bit codes [B, H, N, d] inside
+// the workspace, box {d, 128, 1, 1}: 128-byte swizzle at d = 128, 64-byte
+// swizzle at d = 64 (the swizzle spans one d-byte row).
+dit_status encode_u8_map(CUtensorMap* map, const void* base, int B, int H, int N, int d) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return DIT_ERR_CUDA;
-    const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
-    const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(N) * 128, static_cast<cuuint64_t>(H) * N * 128};
-    const cuuint32_t box[4] = {128, 128, 1, 1};
+    const cuuint64_t D = static_cast<cuuint64_t>(d);
+    const cuuint64_t dims[4] = {D, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {D, static_cast<cuuint64_t>(N) * D, static_cast<cuuint64_t>(H) * N * D};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(d), 128, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapSwizzle sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_INVALID_ARG;
 }
 
 // Validation shared by the 8-bit calls (after check_attn_args).
 dit_status check_q8_args(int d, int smooth_k, int pv_mode, const void* ws, size_t ws_bytes, int B, int H, int N) {
-    if (d != 128) return DIT_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return DIT_ERR_UNSUPPORTED;
     if (smooth_k != 0 && smooth_k != 1) return DIT_ERR_INVALID_ARG;
     if (pv_mode != DIT_PV_FP8_E4M3 && pv_mode != DIT_PV_BF16) return DIT_ERR_INVALID_ARG;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DIT_ERR_WORKSPACE;
@@ -238,7 +235,7 @@ dit_status dit_attn_fwd_ex(const void* q, const void* k, const void* v, void* o,
     if ((st = encode_bf16_map(&tv, v, B, H, Nkv, d, kb, kh, kn)) != DIT_OK) return st;
     const float s = scale > 0.f ? scale : default_scale(d);
     const float scale_log2 = static_cast<float>(static_cast<double>(s) * 1.4426950408889634);
-    cudaError_t e = ATTN_BF16_LAUNCH(tq, tk, tv, o, qb, qh, qn, B, H, Nq, Nkv, d, scale_log2, lse, ds->err_word,
+    cudaError_t e = launch_attn_bf16(tq, tk, tv, o, qb, qh, qn, B, H, Nq, Nkv, d, scale_log2, lse, ds->err_word,
                                      static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
@@ -286,20 +283,20 @@ dit_status dit_attn_fwd(const void* q, const void* k, const void* v, void* o, in
     if ((st = encode_bf16_map(&tv, v, B, H, N, d, sb, sh, sn)) != DIT_OK) return st;
     const float s = scale > 0.f ? scale : default_scale(d);
     const float scale_log2 = static_cast<float>(static_cast<double>(s) * 1.4426950408889634);
-    cudaError_t e = ATTN_BF16_LAUNCH(tq, tk, tv, o, sb, sh, sn, B, H, N, N, d, scale_log2, nullptr, ds->err_word,
+    cudaError_t e = launch_attn_bf16(tq, tk, tv, o, sb, sh, sn, B, H, N, N, d, scale_log2, nullptr, ds->err_word,
                                      static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
 size_t dit_attn_q8_workspace_bytes(int B, int H, int N, int d, int pv_mode) {
-    if (B < 1 || H < 1 || N < 1 || d != 128) return 0;
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
     if (pv_mode != DIT_PV_FP8_E4M3 && pv_mode != DIT_PV_BF16) return 0;
     return q8_layout(B, H, N, d, pv_mode == DIT_PV_FP8_E4M3).total;
 }
 
 dit_status dit_attn_q8_workspace_layout(int B, int H, int N, int d, int pv_mode, size_t* offsets) {
     if (!offsets || B < 1 || H < 1 || N < 1) return DIT_ERR_INVALID_ARG;
-    if (d != 128) return DIT_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return DIT_ERR_UNSUPPORTED;
     if (pv_mode != DIT_PV_FP8_E4M3 && pv_mode != DIT_PV_BF16) return DIT_ERR_INVALID_ARG;
     const Q8Layout L = q8_layout(B, H, N, d, pv_mode == DIT_PV_FP8_E4M3);
     const size_t o[8] = {L.q_codes, L.k_codes, L.v_codes, L.q_scale, L.k_scale, L.k_mean, L.v_scale, L.v_inv};
@@ -316,7 +313,7 @@ dit_status dit_attn_q8_quantize(const void* q, const void* k, const void* v, int
     if ((st = check_q8_args(d, smooth_k, pv_mode, workspace, workspace_bytes, B, H, N)) != DIT_OK) return st;
     DeviceState* ds = device_state(&st);
     if (!ds) return st;
-    cudaError_t e = launch_q8_prepass(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_mode == DIT_PV_FP8_E4M3,
+    cudaError_t e = launch_q8_prepass(q, k, v, sb, sh, sn, B, H, N, d, smooth_k, pv_mode == DIT_PV_FP8_E4M3,
                                       static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
@@ -346,7 +343,7 @@ dit_status dit_attn_q8_channel_stats(const void* k, const void* v, int B, int H,
         return DIT_ERR_INVALID_ARG;
     DeviceState* ds = device_state(&st);
     if (!ds) return st;
-    cudaError_t e = launch_q8_slice_stats(k, v, sb, sh, sn, B, H, N, smooth_k, pv_mode == DIT_PV_FP8_E4M3,
+    cudaError_t e = launch_q8_slice_stats(k, v, sb, sh, sn, B, H, N, d, smooth_k, pv_mode == DIT_PV_FP8_E4M3,
                                           static_cast<uint8_t*>(workspace), k_sum, v_amax,
                                           static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
@@ -365,7 +362,7 @@ dit_status dit_attn_q8_quantize_global(const void* q, const void* k, const void*
     if (n_total < N) return DIT_ERR_INVALID_ARG;
     DeviceState* ds = device_state(&st);
     if (!ds) return st;
-    cudaError_t e = launch_q8_quantize_global(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_mode == DIT_PV_FP8_E4M3,
+    cudaError_t e = launch_q8_quantize_global(q, k, v, sb, sh, sn, B, H, N, d, smooth_k, pv_mode == DIT_PV_FP8_E4M3,
                                               k_sum, v_amax, n_total, static_cast<uint8_t*>(workspace),
                                               static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
@@ -390,16 +387,16 @@ dit_status dit_attn_fwd_q8_prequantized(const void* workspace, size_t workspace_
     if (!ds) return st;
     const uint8_t* ws = static_cast<const uint8_t*>(workspace);
     CUtensorMap tq8, tk8, tv;
-    if ((st = encode_u8_map(&tq8, ws + L.q_codes, B, H, N)) != DIT_OK) return st;
-    if ((st = encode_u8_map(&tk8, ws + L.k_codes, B, H, N)) != DIT_OK) return st;
+    if ((st = encode_u8_map(&tq8, ws + L.q_codes, B, H, N, d)) != DIT_OK) return st;
+    if ((st = encode_u8_map(&tk8, ws + L.k_codes, B, H, N, d)) != DIT_OK) return st;
     if (pv_fp8)
-        st = encode_u8_map(&tv, ws + L.v_codes, B, H, N);
+        st = encode_u8_map(&tv, ws + L.v_codes, B, H, N, d);
     else
         st = encode_bf16_map(&tv, v, B, H, N, d, sb, sh, sn);
     if (st != DIT_OK) return st;
     const float sc = scale > 0.f ? scale : default_scale(d);
     const float scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
-    cudaError_t e = launch_attn_q8(tq8, tk8, tv, pv_fp8, ws, L, o, sb, sh, sn, B, H, N, scale_log2, ds->err_word,
+    cudaError_t e = launch_attn_q8(tq8, tk8, tv, pv_fp8, ws, L, o, sb, sh, sn, B, H, N, d, scale_log2, ds->err_word,
                                    static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
@@ -425,19 +422,19 @@ dit_status dit_attn_fwd_q8(const void* q, const void* k, const void* v, void* o,
     DeviceState* ds = device_state(&st);
     if (!ds) return st;
     CUtensorMap tq8, tk8, tv;
-    if ((st = encode_u8_map(&tq8, ws + L.q_codes, B, H, N)) != DIT_OK) return st;
-    if ((st = encode_u8_map(&tk8, ws + L.k_codes, B, H, N)) != DIT_OK) return st;
+    if ((st = encode_u8_map(&tq8, ws + L.q_codes, B, H, N, d)) != DIT_OK) return st;
+    if ((st = encode_u8_map(&tk8, ws + L.k_codes, B, H, N, d)) != DIT_OK) return st;
     if (pv_fp8)
-        st = encode_u8_map(&tv, ws + L.v_codes, B, H, N);
+        st = encode_u8_map(&tv, ws + L.v_codes, B, H, N, d);
     else
         st = encode_bf16_map(&tv, v, B, H, N, d, sb, sh, sn);
     if (st != DIT_OK) return st;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_q8_prepass(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, s);
+    cudaError_t e = launch_q8_prepass(q, k, v, sb, sh, sn, B, H, N, d, smooth_k, pv_fp8, ws, s);
     if (e != cudaSuccess) return DIT_ERR_CUDA;
     const float sc = scale > 0.f ? scale : default_scale(d);
     const float scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
-    e = launch_attn_q8(tq8, tk8, tv, pv_fp8, ws, L, o, sb, sh, sn, B, H, N, scale_log2, ds->err_word, s);
+    e = launch_attn_q8(tq8, tk8, tv, pv_fp8, ws, L, o, sb, sh, sn, B, H, N, d, scale_log2, ds->err_word, s);
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 

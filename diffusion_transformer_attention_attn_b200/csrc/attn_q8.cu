@@ -21,6 +21,10 @@
 //     weights stay in e4m3's normal range.  l sums the fp32 P̃, and the
 //     epilogue multiplies O by v_scale[c] / l;
 //   * bf16 PV: P = 2^(t − m), threshold 8, as in the bf16 kernel.
+//
+// Head dimension d = 128 or 64.  The 1-byte tiles (Q, K codes and e4m3 V)
+// have d-byte rows: 128-byte swizzle at d = 128, 64-byte swizzle at d = 64;
+// the bf16 V tile is d/64 panels of 64 elements with 128-byte swizzle.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -32,7 +36,6 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int D = 128;
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;
 constexpr int kSoftmaxRegs = 224;
@@ -41,9 +44,9 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchReg
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kPanel = 128 * 128;  // 128 rows × 128 B swizzled panel
+constexpr uint32_t kPanel = 128 * 128;  // 128 rows × 128 B swizzled panel (bf16 V)
 
-template <bool FP8>
+template <bool FP8, int D>
 struct Q8Cfg {
     static constexpr int kQTile = kBM * D;                 // int8
     static constexpr int kKTile = kBN * D;                 // int8
@@ -56,6 +59,9 @@ struct Q8Cfg {
     static constexpr int kNumBars = 1 + 4 * kStages + 6 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;
+    // 1-byte tiles: rows of D bytes, swizzled over D bytes (8-row atoms).
+    static constexpr uint32_t kLayout8 = D == 128 ? kLayoutSw128 : kLayoutSw64;
+    static constexpr uint32_t kAtom8 = 8 * D;  // bytes per 8-row atom
     // Q8·K8ᵀ: s32 accumulate, signed int8 A/B, K-major.
     static constexpr uint32_t kIdescQK = make_idesc(2, 1, 1, 0, 0, 128, kBN);
     // P·V: fp32 accumulate; e4m3 × e4m3 (kind::f8f6f4) or bf16 × bf16, V MN-major.
@@ -69,9 +75,9 @@ struct Bars {
     uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_ready, *mma_done;
 };
 
-template <bool FP8>
+template <bool FP8, int D>
 __device__ __forceinline__ Bars carve(uint8_t* base) {
-    using C = Q8Cfg<FP8>;
+    using C = Q8Cfg<FP8, D>;
     uint64_t* b = reinterpret_cast<uint64_t*>(base + C::kBarOff);
     Bars r;
     r.q_full = b;
@@ -95,17 +101,17 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
     return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-template <bool FP8>
+template <bool FP8, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_q8_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const float* __restrict__ q_scale,
                        const float* __restrict__ k_scale, const float* __restrict__ v_scale,
                        __nv_bfloat16* __restrict__ o, int64_t sb, int64_t sh, int64_t sn, int H, int N, int n_pairs,
                        float scale_log2, int* err) {
-    using C = Q8Cfg<FP8>;
+    using C = Q8Cfg<FP8, D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const Bars bars = carve<FP8>(smem);
+    const Bars bars = carve<FP8, D>(smem);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
@@ -177,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (FP8) {
                         tma_load_4d(smem + C::kVOff + s * C::kVTile, &tv, &bars.v_full[s], 0, j * kBN, h, b);
                     } else {
-                        for (int hf = 0; hf < 2; ++hf)
+                        for (int hf = 0; hf < D / 64; ++hf)
                             tma_load_4d(smem + C::kVOff + s * C::kVTile + hf * kPanel, &tv, &bars.v_full[s], hf * 64,
                                         j * kBN, h, b);
                     }
@@ -195,18 +201,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (warp == kMmaWarp) {
             // -------------------------------------------------------- MMA issuer
             // Descriptors are built once and advanced by byte offsets (SDesc).
-            // K-major int8 operand: k-step kk = 32 bytes inside the 128-B row.
-            // V, MN-major: FP8 rows are one 128-B panel (k-step 32 keys);
-            // bf16 is two 64-element panels 16 KB apart (k-step 16 keys).
-            const SDesc dQ0 = sdesc_sw128(smem_base + C::kQOff, 16, 1024);
+            // K-major int8 operand: k-step kk = 32 bytes inside the D-byte
+            // swizzled row (SBO = one 8-row atom).
+            // V, MN-major: FP8 rows are one D-byte swizzled panel (k-step 32
+            // keys, SBO = one 8-key atom); bf16 is D/64 panels of 64
+            // elements, 16 KB apart (LBO), with 128-byte swizzle (k-step 16 keys).
+            const SDesc dQ0 = sdesc(smem_base + C::kQOff, 16, C::kAtom8, C::kLayout8);
             const SDesc dQ1 = sdesc_add(dQ0, C::kQTile);
-            const SDesc dK0 = sdesc_sw128(smem_base + C::kKOff, 16, 1024);
-            const SDesc dV0 = sdesc_sw128(smem_base + C::kVOff, kPanel, 1024);
+            const SDesc dK0 = sdesc(smem_base + C::kKOff, 16, C::kAtom8, C::kLayout8);
+            const SDesc dV0 = FP8 ? sdesc(smem_base + C::kVOff, kPanel, C::kAtom8, C::kLayout8)
+                                  : sdesc_sw128(smem_base + C::kVOff, kPanel, 1024);
             const uint32_t tS0 = tmem, tS1 = tmem + 128;
-            const uint32_t tO0 = tmem + 256, tO1 = tmem + 384;
+            const uint32_t tO0 = tmem + 256, tO1 = tmem + 256 + D;
             constexpr int kQKSteps = D / 32;
             constexpr int kPVSteps = FP8 ? kBN / 32 : kBN / 16;
-            constexpr uint32_t kVStep = FP8 ? 32 * 128 : 16 * 128;
+            constexpr uint32_t kVStep = FP8 ? 32 * D : 16 * 128;
             auto issue_s = [&](uint32_t tS, SDesc dQ, SDesc dK) {
 #pragma unroll
                 for (int kk = 0; kk < kQKSteps; ++kk)
@@ -450,22 +459,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <bool FP8>
+template <bool FP8, int D>
 cudaError_t launch_mode(const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv, const uint8_t* ws,
                         const Q8Layout& L, void* o, int64_t sb, int64_t sh, int64_t sn, int B, int H, int N,
                         float scale_log2, int* err, cudaStream_t stream) {
-    using C = Q8Cfg<FP8>;
+    using C = Q8Cfg<FP8, D>;
     static_assert(C::kSmemBytes <= 232448, "shared memory budget");
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_q8_kernel<FP8>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_q8_kernel<FP8, D>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(attn_fwd_q8_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    e = cudaFuncSetAttribute(attn_fwd_q8_kernel<FP8, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int n_pairs = ((N + kBM - 1) / kBM + 1) / 2;
     const int64_t grid = static_cast<int64_t>(B) * H * n_pairs;
     if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    attn_fwd_q8_kernel<FP8><<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(
+    attn_fwd_q8_kernel<FP8, D><<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(
         tq8, tk8, tv, reinterpret_cast<const float*>(ws + L.q_scale), reinterpret_cast<const float*>(ws + L.k_scale),
         reinterpret_cast<const float*>(ws + L.v_scale), static_cast<__nv_bfloat16*>(o), sb, sh, sn, H, N, n_pairs,
         scale_log2, err);
@@ -476,9 +485,16 @@ cudaError_t launch_mode(const CUtensorMap& tq8, const CUtensorMap& tk8, const CU
 
 cudaError_t launch_attn_q8(const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv, int pv_fp8,
                            const uint8_t* ws, const Q8Layout& L, void* o, int64_t sb, int64_t sh, int64_t sn, int B,
-                           int H, int N, float scale_log2, int* err, cudaStream_t stream) {
-    if (pv_fp8) return launch_mode<true>(tq8, tk8, tv, ws, L, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
-    return launch_mode<false>(tq8, tk8, tv, ws, L, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
+                           int H, int N, int d, float scale_log2, int* err, cudaStream_t stream) {
+    if (d == 128) {
+        if (pv_fp8) return launch_mode<true, 128>(tq8, tk8, tv, ws, L, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
+        return launch_mode<false, 128>(tq8, tk8, tv, ws, L, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
+    }
+    if (d == 64) {
+        if (pv_fp8) return launch_mode<true, 64>(tq8, tk8, tv, ws, L, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
+        return launch_mode<false, 64>(tq8, tk8, tv, ws, L, o, sb, sh, sn, B, H, N, scale_log2, err, stream);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace ditk

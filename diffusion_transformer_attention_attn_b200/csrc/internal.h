@@ -18,12 +18,6 @@ cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const
                              int64_t sb, int64_t sh, int64_t sn, int B, int H, int Nq, int Nkv, int d,
                              float scale_log2, float* lse, int* err, cudaStream_t stream);
 
-// The same attention with one 128-row query tile per CTA and the keys of each
-// tile split between two softmax warpgroups (attn_bf16_ks.cu).
-cudaError_t launch_attn_bf16_ks(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                                int64_t sb, int64_t sh, int64_t sn, int B, int H, int Nq, int Nkv, int d,
-                                float scale_log2, float* lse, int* err, cudaStream_t stream);
-
 // Bounded-wait self-test (selftest.cu): one warp waits on an mbarrier that is
 // never arrived on, gives up after the wait limit and records DIT_ERR_TIMEOUT
 // in *err; *completed gets 0 (1 would mean the wait ended normally).
@@ -35,7 +29,7 @@ cudaError_t launch_attn_merge(const void* const* o_parts, const float* const* ls
                               int N, int d, int64_t sb, int64_t sh, int64_t sn, void* o, float* lse,
                               cudaStream_t stream);
 
-// ---- 8-bit path (d = 128) ----------------------------------------------
+// ---- 8-bit path (d = 64 or 128) ---------------------------------------
 // Tokens per statistics chunk of the pre-pass.
 constexpr int kQ8StatChunk = 256;
 
@@ -51,27 +45,29 @@ Q8Layout q8_layout(int B, int H, int N, int d, int pv_fp8);
 
 // Statistics and quantisation of Q, K (and V when pv_fp8) into `ws`.
 cudaError_t launch_q8_prepass(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
-                              int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream);
+                              int H, int N, int d, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream);
 
 // The quantisation launches of the pre-pass alone (K mean and V scales
 // already in `ws`).
 cudaError_t launch_q8_codes(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
-                            int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream);
+                            int H, int N, int d, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream);
 // Token-sharded pre-pass: the slice's per-channel K sums (fp64) and V maxima,
 // then quantisation with the statistics combined over n_total tokens.
 cudaError_t launch_q8_slice_stats(const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H,
-                                  int N, int smooth_k, int pv_fp8, uint8_t* ws, double* k_sum, float* v_amax,
+                                  int N, int d, int smooth_k, int pv_fp8, uint8_t* ws, double* k_sum, float* v_amax,
                                   cudaStream_t stream);
 cudaError_t launch_q8_quantize_global(const void* q, const void* k, const void* v, int64_t sb, int64_t sh,
-                                      int64_t sn, int B, int H, int N, int smooth_k, int pv_fp8, const double* k_sum,
-                                      const float* v_amax, int64_t n_total, uint8_t* ws, cudaStream_t stream);
+                                      int64_t sn, int B, int H, int N, int d, int smooth_k, int pv_fp8,
+                                      const double* k_sum, const float* v_amax, int64_t n_total, uint8_t* ws,
+                                      cudaStream_t stream);
 
 // 8-bit attention over the pre-pass products.  tq8/tk8: 4-D maps over the
-// INT8 codes {d, N, H, B}, box {128, 128, 1, 1}; tv: e4m3 codes (same box,
-// pv_fp8) or the caller's bf16 V (box {64, 128, 1, 1}).
+// INT8 codes {d, N, H, B}, box {d, 128, 1, 1} (128-byte swizzle at d = 128,
+// 64-byte at d = 64); tv: e4m3 codes (same box and swizzle, pv_fp8) or the
+// caller's bf16 V (box {64, 128, 1, 1}, 128-byte swizzle).
 cudaError_t launch_attn_q8(const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv, int pv_fp8,
                            const uint8_t* ws, const Q8Layout& L, void* o, int64_t sb, int64_t sh, int64_t sn, int B,
-                           int H, int N, float scale_log2, int* err, cudaStream_t stream);
+                           int H, int N, int d, float scale_log2, int* err, cudaStream_t stream);
 
 // DIT_OK when the current device is an sm_100 part (its one-time set-up done),
 // else DIT_ERR_UNSUPPORTED or DIT_ERR_CUDA.

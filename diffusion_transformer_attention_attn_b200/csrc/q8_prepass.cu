@@ -7,12 +7,15 @@
 //   * Q: INT8 per block of 128 tokens (all d channels): amax over the block's
 //     valid tokens, inv = 127/amax and scale = amax/127 (fp32 divisions),
 //     code = round-half-even(x·inv) saturated to ±127.  amax = 0 gives
-//     scale = inv = 0 and all-zero codes (no NaN).
+//     scale = inv = 0 and all-zero codes (no NaN); so does an amax so small
+//     that 127/amax overflows fp32 (below about 3.7e-37), whose block would
+//     otherwise turn its exact zeros into 0·inf = NaN.
 //   * K: optionally minus its per-channel mean over all N tokens (this shifts
 //     every logit of a query row by the same amount, so softmax is unchanged),
 //     then INT8 per block of 64 tokens as above.
 //   * V (FP8 PV only): per channel, amax over all N tokens, scale = amax/448,
-//     code = e4m3(x·448/amax), round to nearest even, saturating; same guard.
+//     code = e4m3(x·448/amax), round to nearest even, saturating; same guard
+//     (amax zero, or 448/amax not finite).
 //
 // Token-sharded form (launch_q8_slice_stats, launch_q8_quantize_global): each
 // device reduces its token slice to per-channel K sums and V maxima, the
@@ -20,6 +23,8 @@
 // combined statistics, so that the 1-byte codes, not the bf16 values, travel
 // in a Ulysses all-to-all.
 //
+// Head dimension d = 128 or 64 (a template argument of every kernel; a
+// thread always covers 8 consecutive channels, one 16-byte load per row).
 // Three launches, each HBM-bound with 16-byte vector loads:
 //   q8_stats_kernel     per (b,h) and chunk of 256 tokens: fp64 column sums of
 //                       K and column |V| maxima -> partials
@@ -55,18 +60,20 @@ __device__ __forceinline__ const uint4* row_ptr(const void* base, int64_t sb, in
     return reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + b * sb + h * sh + n * sn);
 }
 
-// grid (n_chunks, B*H).  Thread t: 8 channels [8·(t%16), +8), rows t/16 + 16·i.
-// Four blocks per SM (64 registers) keep more loads in flight than two
-// blocks with deeper per-thread batches.
+// grid (n_chunks, B*H).  With G = D/8 channel groups, thread t holds channels
+// [8·(t%G), +8) of rows t/G + (256/G)·i.  Four blocks per SM (64 registers)
+// keep more loads in flight than two blocks with deeper per-thread batches.
+template <int D>
 __global__ void __launch_bounds__(kStatThreads, 4)
     q8_stats_kernel(const void* __restrict__ k, const void* __restrict__ v, int64_t sb, int64_t sh, int64_t sn, int H,
                     int N, int chunk, int want_sum, int want_vmax, double* __restrict__ psum,
                     float* __restrict__ pmax) {
-    constexpr int D = 128;
-    __shared__ double s_sum[kStatThreads / 16][D];
-    __shared__ float s_max[kStatThreads / 16][D];
+    constexpr int kCG = D / 8;                  // channel groups per row
+    constexpr int kStep = kStatThreads / kCG;   // rows between a thread's rows
+    __shared__ double s_sum[kStep][D];
+    __shared__ float s_max[kStep][D];
     const int bh = blockIdx.y, b = bh / H, h = bh % H;
-    const int cg = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+    const int cg = threadIdx.x % kCG, r0 = threadIdx.x / kCG;
     const int64_t n0 = static_cast<int64_t>(blockIdx.x) * chunk;
     const int64_t n1 = min(static_cast<int64_t>(N), n0 + chunk);
     double acc[8];
@@ -78,7 +85,6 @@ __global__ void __launch_bounds__(kStatThreads, 4)
     }
     // Rows are visited in the same order as one at a time, but the loads of
     // kBatch rows are issued before any of them is used.
-    constexpr int kStep = kStatThreads / 16;  // rows between a thread's rows
     constexpr int kBatch = 2;
     for (int64_t nb = n0 + r0; nb < n1; nb += kBatch * kStep) {
         uint4 kr[kBatch], vr[kBatch];
@@ -117,7 +123,7 @@ __global__ void __launch_bounds__(kStatThreads, 4)
         const int c = threadIdx.x;
         double s = 0.0;
         float m = 0.f;
-        for (int r = 0; r < kStatThreads / 16; ++r) {
+        for (int r = 0; r < kStep; ++r) {
             s += s_sum[r][c];
             m = fmaxf(m, s_max[r][c]);
         }
@@ -128,17 +134,17 @@ __global__ void __launch_bounds__(kStatThreads, 4)
 }
 
 // Per (b,h) and channel: the partials' K sum and V maximum over all chunks.
-// kFinGroups × 128 threads; group g takes chunks g, g + kFinGroups, ... in
+// kFinGroups × D threads; group g takes chunks g, g + kFinGroups, ... in
 // order, then thread (0, c) adds the groups' sums in group order, so the
 // result does not depend on timing.  Only group 0's (sum, max) are complete.
 constexpr int kFinGroups = 8;
+template <int D>
 __device__ __forceinline__ void chunk_reduce(const double* __restrict__ psum, const float* __restrict__ pmax,
                                              int n_chunks, int want_sum, int want_vmax, double& s_out,
                                              float& m_out) {
-    constexpr int D = 128;
     __shared__ double s_part[kFinGroups][D];
     __shared__ float m_part[kFinGroups][D];
-    const int bh = blockIdx.x, c = threadIdx.x & (D - 1), g = threadIdx.x / D;
+    const int bh = blockIdx.x, c = threadIdx.x % D, g = threadIdx.x / D;
     double s = 0.0;
     float m = 0.f;
     for (int i = g; i < n_chunks; i += kFinGroups) {
@@ -159,24 +165,34 @@ __device__ __forceinline__ void chunk_reduce(const double* __restrict__ psum, co
     m_out = m;
 }
 
-// grid B*H, kFinGroups × 128 threads.
-__global__ void __launch_bounds__(kFinGroups * 128)
+// V's per-channel scale and its inverse from the channel's |V| maximum, with
+// the zero-scale guard: a maximum of zero, or one whose inverse 448/m is not
+// a finite fp32 number, gives scale = inv = 0 (zero codes, no NaN).
+__device__ __forceinline__ void v_scales(float m, float& sc, float& inv) {
+    sc = 0.f;
+    inv = 0.f;
+    const float i = __fdiv_rn(448.f, m);
+    if (m > 0.f && isfinite(i)) {
+        sc = __fdiv_rn(m, 448.f);
+        inv = i;
+    }
+}
+
+// grid B*H, kFinGroups × D threads.
+template <int D>
+__global__ void __launch_bounds__(kFinGroups * D)
     q8_finalize_kernel(const double* __restrict__ psum, const float* __restrict__ pmax, int n_chunks, int N,
                        int want_sum, int want_vmax, float* __restrict__ k_mean, float* __restrict__ v_scale,
                        float* __restrict__ v_inv) {
-    constexpr int D = 128;
     const int bh = blockIdx.x, c = threadIdx.x;
     double s;
     float m;
-    chunk_reduce(psum, pmax, n_chunks, want_sum, want_vmax, s, m);
+    chunk_reduce<D>(psum, pmax, n_chunks, want_sum, want_vmax, s, m);
     if (threadIdx.x >= D) return;
     k_mean[bh * D + c] = want_sum ? static_cast<float>(s / static_cast<double>(N)) : 0.f;
     if (want_vmax) {
-        float sc = 0.f, inv = 0.f;
-        if (m > 0.f) {  // zero-scale guard
-            sc = __fdiv_rn(m, 448.f);
-            inv = __fdiv_rn(448.f, m);
-        }
+        float sc, inv;
+        v_scales(m, sc, inv);
         v_scale[bh * D + c] = sc;
         v_inv[bh * D + c] = inv;
     }
@@ -193,19 +209,21 @@ __device__ __forceinline__ uint32_t s8x4(float a, float b, float c, float d) {
 }
 
 // INT8 per block of BLK tokens.  grid (ceil(N/BLK), B*H), THREADS threads:
-// thread t holds channels [8·(t%16), +8) of rows t/16 + (THREADS/16)·i of
-// the block (Q: 128 tokens on 512 threads, K: 64 tokens on 256 threads).
+// with G = D/8, thread t holds channels [8·(t%G), +8) of rows t/G +
+// (THREADS/G)·i of the block (d = 128: Q 128 tokens on 512 threads, K 64
+// tokens on 256; d = 64: half the threads; four rows per thread throughout).
 // Codes are cvt.rni.sat.s8.f32 of x·inv: round half to even, saturated.
-template <int BLK, int THREADS>
+template <int D, int BLK, int THREADS>
 __global__ void __launch_bounds__(THREADS, 1536 / THREADS)
     q8_quant_int8_kernel(const void* __restrict__ x, int64_t sb, int64_t sh, int64_t sn, int H, int N,
                          const float* __restrict__ mean, int8_t* __restrict__ codes, float* __restrict__ scales) {
-    constexpr int D = 128;
-    constexpr int kGroups = THREADS / 16;  // row groups
-    constexpr int kRows = BLK / kGroups;   // rows per thread
+    constexpr int kCG = D / 8;
+    constexpr int kGroups = THREADS / kCG;  // row groups
+    constexpr int kRows = BLK / kGroups;    // rows per thread
+    static_assert(kRows * kGroups == BLK, "rows per thread");
     __shared__ float s_red[THREADS / 32];
     const int bh = blockIdx.y, b = bh / H, h = bh % H;
-    const int cg = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+    const int cg = threadIdx.x % kCG, r0 = threadIdx.x / kCG;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * BLK;
     float mu[8];
 #pragma unroll
@@ -237,9 +255,11 @@ __global__ void __launch_bounds__(THREADS, 1536 / THREADS)
     amax = s_red[0];
 #pragma unroll
     for (int w = 1; w < THREADS / 32; ++w) amax = fmaxf(amax, s_red[w]);
+    // Zero-scale guard: amax zero, or so small that 127/amax is not finite.
     float inv = 0.f, scale = 0.f;
-    if (amax > 0.f) {  // zero-scale guard
-        inv = __fdiv_rn(127.f, amax);
+    const float inv_raw = __fdiv_rn(127.f, amax);
+    if (amax > 0.f && isfinite(inv_raw)) {
+        inv = inv_raw;
         scale = __fdiv_rn(amax, 127.f);
     }
     if (threadIdx.x == 0) scales[static_cast<int64_t>(bh) * gridDim.x + blockIdx.x] = scale;
@@ -266,20 +286,23 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
     return r;
 }
 
-// FP8 e4m3 per channel.  grid (ceil(N/128), B*H), 256 threads, as above.
+// FP8 e4m3 per channel.  grid (ceil(N/128), B*H), 256 threads; thread t
+// holds channels [8·(t%G), +8) of rows t/G + (256/G)·i of the 128-row block.
+template <int D>
 __global__ void __launch_bounds__(kQuantThreads)
     q8_quant_e4m3_kernel(const void* __restrict__ x, int64_t sb, int64_t sh, int64_t sn, int H, int N,
                          const float* __restrict__ v_inv, uint8_t* __restrict__ codes) {
-    constexpr int D = 128;
+    constexpr int kCG = D / 8;
+    constexpr int kStep = kQuantThreads / kCG;
     const int bh = blockIdx.y, b = bh / H, h = bh % H;
-    const int cg = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+    const int cg = threadIdx.x % kCG, r0 = threadIdx.x / kCG;
     float inv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) inv[i] = v_inv[bh * D + cg * 8 + i];
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * 128;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int64_t n = t0 + r0 + 16 * r;
+    for (int r = 0; r < 128 / kStep; ++r) {
+        const int64_t n = t0 + r0 + kStep * r;
         if (n < N) {
             float f[8];
             unpack8(__ldg(row_ptr(x, sb, sh, sn, b, h, n) + cg), f);
@@ -295,38 +318,102 @@ __global__ void __launch_bounds__(kQuantThreads)
 
 // Token-sharded form (one slice of the tokens per device): the per-channel
 // K sums and V maxima of this slice, for the devices to combine.  grid B*H,
-// kFinGroups × 128 threads; the same fixed-order sum as q8_finalize.
-__global__ void __launch_bounds__(kFinGroups * 128)
+// kFinGroups × D threads; the same fixed-order sum as q8_finalize.
+template <int D>
+__global__ void __launch_bounds__(kFinGroups * D)
     q8_slice_stats_kernel(const double* __restrict__ psum, const float* __restrict__ pmax, int n_chunks,
                           int want_sum, int want_vmax, double* __restrict__ k_sum, float* __restrict__ v_amax) {
-    constexpr int D = 128;
     const int bh = blockIdx.x, c = threadIdx.x;
     double s;
     float m;
-    chunk_reduce(psum, pmax, n_chunks, want_sum, want_vmax, s, m);
+    chunk_reduce<D>(psum, pmax, n_chunks, want_sum, want_vmax, s, m);
     if (threadIdx.x >= D) return;
     k_sum[bh * D + c] = s;
     v_amax[bh * D + c] = m;
 }
 
 // The K mean and V scales from the combined statistics of all slices
-// (n_total tokens): the arithmetic of q8_finalize_kernel.
+// (n_total tokens): the arithmetic of q8_finalize_kernel.  D threads.
+template <int D>
 __global__ void q8_finalize_global_kernel(const double* __restrict__ k_sum, const float* __restrict__ v_amax,
                                           int64_t n_total, int want_sum, int want_vmax, float* __restrict__ k_mean,
                                           float* __restrict__ v_scale, float* __restrict__ v_inv) {
-    constexpr int D = 128;
     const int bh = blockIdx.x, c = threadIdx.x;
     k_mean[bh * D + c] = want_sum ? static_cast<float>(k_sum[bh * D + c] / static_cast<double>(n_total)) : 0.f;
     if (want_vmax) {
-        const float m = v_amax[bh * D + c];
-        float sc = 0.f, inv = 0.f;
-        if (m > 0.f) {  // zero-scale guard
-            sc = __fdiv_rn(m, 448.f);
-            inv = __fdiv_rn(448.f, m);
-        }
+        float sc, inv;
+        v_scales(v_amax[bh * D + c], sc, inv);
         v_scale[bh * D + c] = sc;
         v_inv[bh * D + c] = inv;
     }
+}
+
+template <int D>
+cudaError_t prepass_d(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H,
+                      int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
+    const Q8Layout L = q8_layout(B, H, N, D, pv_fp8);
+    double* psum = reinterpret_cast<double*>(ws + L.psum);
+    float* pmax = reinterpret_cast<float*>(ws + L.pmax);
+    const int BH = B * H;
+    if (smooth_k || pv_fp8) {
+        q8_stats_kernel<D><<<dim3(L.n_chunks, BH), kStatThreads, 0, stream>>>(k, v, sb, sh, sn, H, N, kQ8StatChunk,
+                                                                              smooth_k, pv_fp8, psum, pmax);
+        q8_finalize_kernel<D><<<BH, kFinGroups * D, 0, stream>>>(psum, pmax, L.n_chunks, N, smooth_k, pv_fp8,
+                                                                 reinterpret_cast<float*>(ws + L.k_mean),
+                                                                 reinterpret_cast<float*>(ws + L.v_scale),
+                                                                 reinterpret_cast<float*>(ws + L.v_inv));
+    }
+    return launch_q8_codes(q, k, v, sb, sh, sn, B, H, N, D, smooth_k, pv_fp8, ws, stream);
+}
+
+template <int D>
+cudaError_t codes_d(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H,
+                    int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
+    const Q8Layout L = q8_layout(B, H, N, D, pv_fp8);
+    const int BH = B * H;
+    const float* k_mean = reinterpret_cast<const float*>(ws + L.k_mean);
+    const float* v_inv = reinterpret_cast<const float*>(ws + L.v_inv);
+    // Four rows per thread in both quantisers and at both head sizes.
+    constexpr int kQThreads = 4 * D, kKThreads = 2 * D;
+    q8_quant_int8_kernel<D, 128, kQThreads><<<dim3((N + 127) / 128, BH), kQThreads, 0, stream>>>(
+        q, sb, sh, sn, H, N, nullptr, reinterpret_cast<int8_t*>(ws + L.q_codes),
+        reinterpret_cast<float*>(ws + L.q_scale));
+    q8_quant_int8_kernel<D, 64, kKThreads><<<dim3((N + 63) / 64, BH), kKThreads, 0, stream>>>(
+        k, sb, sh, sn, H, N, smooth_k ? k_mean : nullptr, reinterpret_cast<int8_t*>(ws + L.k_codes),
+        reinterpret_cast<float*>(ws + L.k_scale));
+    if (pv_fp8)
+        q8_quant_e4m3_kernel<D><<<dim3((N + 127) / 128, BH), kQuantThreads, 0, stream>>>(v, sb, sh, sn, H, N, v_inv,
+                                                                                         ws + L.v_codes);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t slice_stats_d(const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H, int N,
+                          int smooth_k, int pv_fp8, uint8_t* ws, double* k_sum, float* v_amax, cudaStream_t stream) {
+    const Q8Layout L = q8_layout(B, H, N, D, pv_fp8);
+    const int BH = B * H;
+    double* psum = reinterpret_cast<double*>(ws + L.psum);
+    float* pmax = reinterpret_cast<float*>(ws + L.pmax);
+    if (smooth_k || pv_fp8)
+        q8_stats_kernel<D><<<dim3(L.n_chunks, BH), kStatThreads, 0, stream>>>(k, v, sb, sh, sn, H, N, kQ8StatChunk,
+                                                                              smooth_k, pv_fp8, psum, pmax);
+    q8_slice_stats_kernel<D><<<BH, kFinGroups * D, 0, stream>>>(psum, pmax, L.n_chunks, smooth_k, pv_fp8, k_sum,
+                                                                v_amax);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t quantize_global_d(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
+                              int H, int N, int smooth_k, int pv_fp8, const double* k_sum, const float* v_amax,
+                              int64_t n_total, uint8_t* ws, cudaStream_t stream) {
+    const Q8Layout L = q8_layout(B, H, N, D, pv_fp8);
+    q8_finalize_global_kernel<D><<<B * H, D, 0, stream>>>(k_sum, v_amax, n_total, smooth_k, pv_fp8,
+                                                          reinterpret_cast<float*>(ws + L.k_mean),
+                                                          reinterpret_cast<float*>(ws + L.v_scale),
+                                                          reinterpret_cast<float*>(ws + L.v_inv));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_q8_codes(q, k, v, sb, sh, sn, B, H, N, D, smooth_k, pv_fp8, ws, stream);
 }
 
 }  // namespace
@@ -353,66 +440,38 @@ Q8Layout q8_layout(int B, int H, int N, int d, int pv_fp8) {
 }
 
 cudaError_t launch_q8_prepass(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
-                              int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
-    const Q8Layout L = q8_layout(B, H, N, 128, pv_fp8);
-    double* psum = reinterpret_cast<double*>(ws + L.psum);
-    float* pmax = reinterpret_cast<float*>(ws + L.pmax);
-    float* k_mean = reinterpret_cast<float*>(ws + L.k_mean);
-    float* v_scale = reinterpret_cast<float*>(ws + L.v_scale);
-    float* v_inv = reinterpret_cast<float*>(ws + L.v_inv);
-    const int BH = B * H;
-    if (smooth_k || pv_fp8) {
-        q8_stats_kernel<<<dim3(L.n_chunks, BH), kStatThreads, 0, stream>>>(k, v, sb, sh, sn, H, N, kQ8StatChunk,
-                                                                           smooth_k, pv_fp8, psum, pmax);
-        q8_finalize_kernel<<<BH, kFinGroups * 128, 0, stream>>>(psum, pmax, L.n_chunks, N, smooth_k, pv_fp8, k_mean, v_scale,
-                                                   v_inv);
-    }
-    return launch_q8_codes(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, stream);
+                              int H, int N, int d, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
+    if (d == 128) return prepass_d<128>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, stream);
+    if (d == 64) return prepass_d<64>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, stream);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_q8_codes(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
-                            int H, int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
-    const Q8Layout L = q8_layout(B, H, N, 128, pv_fp8);
-    const int BH = B * H;
-    const float* k_mean = reinterpret_cast<const float*>(ws + L.k_mean);
-    const float* v_inv = reinterpret_cast<const float*>(ws + L.v_inv);
-    q8_quant_int8_kernel<128, 512><<<dim3((N + 127) / 128, BH), 512, 0, stream>>>(
-        q, sb, sh, sn, H, N, nullptr, reinterpret_cast<int8_t*>(ws + L.q_codes),
-        reinterpret_cast<float*>(ws + L.q_scale));
-    q8_quant_int8_kernel<64, 256><<<dim3((N + 63) / 64, BH), 256, 0, stream>>>(
-        k, sb, sh, sn, H, N, smooth_k ? k_mean : nullptr, reinterpret_cast<int8_t*>(ws + L.k_codes),
-        reinterpret_cast<float*>(ws + L.k_scale));
-    if (pv_fp8)
-        q8_quant_e4m3_kernel<<<dim3((N + 127) / 128, BH), kQuantThreads, 0, stream>>>(
-            v, sb, sh, sn, H, N, v_inv, ws + L.v_codes);
-    return cudaGetLastError();
+                            int H, int N, int d, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
+    if (d == 128) return codes_d<128>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, stream);
+    if (d == 64) return codes_d<64>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, stream);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_q8_slice_stats(const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H,
-                                  int N, int smooth_k, int pv_fp8, uint8_t* ws, double* k_sum, float* v_amax,
+                                  int N, int d, int smooth_k, int pv_fp8, uint8_t* ws, double* k_sum, float* v_amax,
                                   cudaStream_t stream) {
-    const Q8Layout L = q8_layout(B, H, N, 128, pv_fp8);
-    const int BH = B * H;
-    double* psum = reinterpret_cast<double*>(ws + L.psum);
-    float* pmax = reinterpret_cast<float*>(ws + L.pmax);
-    if (smooth_k || pv_fp8)
-        q8_stats_kernel<<<dim3(L.n_chunks, BH), kStatThreads, 0, stream>>>(k, v, sb, sh, sn, H, N, kQ8StatChunk,
-                                                                           smooth_k, pv_fp8, psum, pmax);
-    q8_slice_stats_kernel<<<BH, kFinGroups * 128, 0, stream>>>(psum, pmax, L.n_chunks, smooth_k, pv_fp8, k_sum, v_amax);
-    return cudaGetLastError();
+    if (d == 128) return slice_stats_d<128>(k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, k_sum, v_amax, stream);
+    if (d == 64) return slice_stats_d<64>(k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, k_sum, v_amax, stream);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_q8_quantize_global(const void* q, const void* k, const void* v, int64_t sb, int64_t sh,
-                                      int64_t sn, int B, int H, int N, int smooth_k, int pv_fp8, const double* k_sum,
-                                      const float* v_amax, int64_t n_total, uint8_t* ws, cudaStream_t stream) {
-    const Q8Layout L = q8_layout(B, H, N, 128, pv_fp8);
-    q8_finalize_global_kernel<<<B * H, 128, 0, stream>>>(k_sum, v_amax, n_total, smooth_k, pv_fp8,
-                                                         reinterpret_cast<float*>(ws + L.k_mean),
-                                                         reinterpret_cast<float*>(ws + L.v_scale),
-                                                         reinterpret_cast<float*>(ws + L.v_inv));
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    return launch_q8_codes(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, stream);
+                                      int64_t sn, int B, int H, int N, int d, int smooth_k, int pv_fp8,
+                                      const double* k_sum, const float* v_amax, int64_t n_total, uint8_t* ws,
+                                      cudaStream_t stream) {
+    if (d == 128)
+        return quantize_global_d<128>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, k_sum, v_amax, n_total, ws,
+                                      stream);
+    if (d == 64)
+        return quantize_global_d<64>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, k_sum, v_amax, n_total, ws,
+                                     stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace ditk

@@ -161,16 +161,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 // Shared-memory matrix descriptor (tcgen05 "matrix descriptor" format):
 //   bits  0-13 start address >> 4       bits 16-29 leading byte offset >> 4
 //   bits 32-45 stride byte offset >> 4  bits 46-47 version (1 on sm_100)
-//   bits 49-51 base offset (0: atoms 1024-B aligned)
-//   bits 61-63 layout: 2 = 128-byte swizzle
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+//   bits 49-51 base offset (0: atoms aligned to their own size)
+//   bits 61-63 layout: 2 = 128-byte swizzle (8 rows × 128 B atoms),
+//                      4 = 64-byte swizzle (8 rows × 64 B atoms)
+constexpr uint32_t kLayoutSw128 = 2;
+constexpr uint32_t kLayoutSw64 = 4;
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
     d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
     d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= 1ull << 46;
-    d |= 2ull << 61;
+    d |= static_cast<uint64_t>(layout & 7u) << 61;
     return d;
+}
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return smem_desc(saddr, lbo_bytes, sbo_bytes, kLayoutSw128);
 }
 
 // Instruction descriptor for kind::f16 / kind::i8 / kind::f8f6f4 (dense):
@@ -192,9 +199,12 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t dfmt, uint32_t afmt, 
 struct SDesc {
     uint32_t lo, hi;
 };
-__device__ __forceinline__ SDesc sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-    const uint64_t d = smem_desc_sw128(saddr, lbo_bytes, sbo_bytes);
+__device__ __forceinline__ SDesc sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes, uint32_t layout) {
+    const uint64_t d = smem_desc(saddr, lbo_bytes, sbo_bytes, layout);
     return SDesc{static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
+}
+__device__ __forceinline__ SDesc sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return sdesc(saddr, lbo_bytes, sbo_bytes, kLayoutSw128);
 }
 __device__ __forceinline__ SDesc sdesc_add(SDesc d, uint32_t bytes) { return SDesc{d.lo + (bytes >> 4), d.hi}; }
 

@@ -130,8 +130,9 @@ dit_status dit_attn_merge(const void* const* o_parts, const float* const* lse_pa
  *         a per-row logit shift, so the softmax is unchanged), then INT8 per
  *         block of 64 tokens;
  *   INT8 scales: amax over the block's valid tokens, scale = amax/127,
- *         codes = round-half-even(x·127/amax) in [-127, 127]; amax = 0 gives
- *         scale 0 and zero codes;
+ *         codes = round-half-even(x·127/amax) in [-127, 127]; amax = 0, or an
+ *         amax so small that 127/amax overflows fp32, gives scale 0 and
+ *         zero codes (V likewise with 448/amax);
  *   S = Q8·K8ᵀ in int32, dequantised by q_scale·k_scale;
  *   P·V in FP8 e4m3 (pv_mode DIT_PV_FP8_E4M3: V per channel, scale
  *         amax/448; P scaled by 2^6.5 before e4m3) or in bf16 (DIT_PV_BF16:
@@ -144,7 +145,7 @@ dit_status dit_attn_merge(const void* const* o_parts, const float* const* lse_pa
  *                   256-byte aligned, not overlapping q, k, v or o; no
  *                   initialisation needed.  It receives the codes and scales
  *                   (layout: dit_attn_q8_workspace_layout).
- *   d must be 128 (others: DIT_ERR_UNSUPPORTED).
+ *   d               64 or 128 (others: DIT_ERR_UNSUPPORTED).
  *   Launches the pre-pass (3-5 kernels) and the attention kernel on `stream`.
  */
 size_t dit_attn_q8_workspace_bytes(int B, int H, int N, int d, int pv_mode);

@@ -112,7 +112,9 @@ def test_product_path_does_not_reach_the_oracle():
 
 
 def test_q8_workspace_size_and_layout(lib):
-    assert lib.dit_attn_q8_workspace_bytes(1, 2, 256, 64, 0) == 0          # d = 64: not served
+    assert lib.dit_attn_q8_workspace_bytes(1, 2, 256, 96, 0) == 0          # d = 96: not served
+    d64 = lib.dit_attn_q8_workspace_bytes(1, 2, 256, 64, 0)                 # d = 64: half the codes
+    assert 3 * 2 * 256 * 64 <= d64 < lib.dit_attn_q8_workspace_bytes(1, 2, 256, 128, 0)
     assert lib.dit_attn_q8_workspace_bytes(1, 2, 256, 128, 7) == 0         # bad mode
     fp8 = lib.dit_attn_q8_workspace_bytes(1, 24, 4608, 128, dit.DIT_PV_FP8_E4M3)
     bf = lib.dit_attn_q8_workspace_bytes(1, 24, 4608, 128, dit.DIT_PV_BF16)
@@ -134,7 +136,7 @@ def _q8(lib, q=Q, k=K, v=V, o=O, B=1, H=2, N=256, d=128, smooth=1, mode=0, ws=WS
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(d=64), dit.DIT_ERR_UNSUPPORTED),
+    (dict(d=96), dit.DIT_ERR_UNSUPPORTED),
     (dict(mode=5), dit.DIT_ERR_INVALID_ARG),
     (dict(smooth=2), dit.DIT_ERR_INVALID_ARG),
     (dict(ws=0), dit.DIT_ERR_WORKSPACE),
@@ -150,7 +152,7 @@ def test_q8_argument_errors(lib, kw, status):
 
 def test_q8_quantize_argument_errors(lib):
     wsb = lib.dit_attn_q8_workspace_bytes(1, 2, 256, 128, 0)
-    assert lib.dit_attn_q8_quantize(Q, K, V, 1, 2, 256, 64, None, 1, 0, WS, wsb, None) == dit.DIT_ERR_UNSUPPORTED
+    assert lib.dit_attn_q8_quantize(Q, K, V, 1, 2, 256, 96, None, 1, 0, WS, wsb, None) == dit.DIT_ERR_UNSUPPORTED
     assert lib.dit_attn_q8_quantize(Q, K, V, 1, 2, 256, 128, None, 1, 0, WS, 100, None) == dit.DIT_ERR_WORKSPACE
     assert lib.dit_attn_q8_quantize(0, K, V, 1, 2, 256, 128, None, 1, 0, WS, wsb, None) == dit.DIT_ERR_INVALID_ARG
 
@@ -290,7 +292,7 @@ def test_sharded_q8_argument_errors(lib):
                                                     kw.get("smooth", 1), kw.get("mode", 0), kw.get("ks", KS),
                                                     kw.get("va", VA), kw.get("ws", WS), kw.get("wsb", wsb), None)
     assert st(k=0) == dit.DIT_ERR_INVALID_ARG
-    assert st(d=64) == dit.DIT_ERR_UNSUPPORTED
+    assert st(d=96) == dit.DIT_ERR_UNSUPPORTED
     assert st(mode=3) == dit.DIT_ERR_INVALID_ARG
     assert st(ks=0) == dit.DIT_ERR_INVALID_ARG
     assert st(ks=KS + 4) == dit.DIT_ERR_INVALID_ARG

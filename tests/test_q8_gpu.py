@@ -62,15 +62,9 @@ def _check(out, ref, mode, what):
 
 # ---------------------------------------------------------------- pre-pass, bit for bit
 
-@pytest.mark.parametrize("case,N,smooth", [
-    (inputs.IMAGE_Q8, 1000, True),
-    (inputs.IMAGE_Q8, 1000, False),
-    (inputs.AttnCase("q8_small", 2, 3, 333, 128, k_offset_std=2.0, seed=21), None, True),
-    (inputs.AttnCase("q8_one", 1, 1, 1, 128, seed=22), None, True),
-])
-def test_prepass_matches_oracle_quantiser(case, N, smooth):
+def _check_prepass(q, k, v, smooth):
+    """The pre-pass products equal the oracle's fp32 quantiser bit for bit."""
     import diffusion_transformer_attention_attn_b200 as dit
-    q, k, v = inputs.attn_inputs(case, N=N)
     B, H, n, d = q.shape
     ws = dit.dit_attn_q8_quantize(*_dev(q, k, v), smooth_k=smooth, pv_mode="fp8")
     torch.cuda.synchronize()
@@ -87,6 +81,57 @@ def test_prepass_matches_oracle_quantiser(case, N, smooth):
     np.testing.assert_array_equal(views["k_codes"], kc)
     np.testing.assert_array_equal(views["v_scale"], vs)
     np.testing.assert_array_equal(views["v_codes"], vc)
+
+
+@pytest.mark.parametrize("case,N,smooth", [
+    (inputs.IMAGE_Q8, 1000, True),
+    (inputs.IMAGE_Q8, 1000, False),
+    (inputs.AttnCase("q8_small", 2, 3, 333, 128, k_offset_std=2.0, seed=21), None, True),
+    (inputs.AttnCase("q8_one", 1, 1, 1, 128, seed=22), None, True),
+    (inputs.AttnCase("q8_d64", 2, 3, 333, 64, k_offset_std=3.0, zero_q_channel=5, zero_q_tokens=(128, 256),
+                     seed=23), None, True),
+    (inputs.AttnCase("q8_d64", 2, 3, 333, 64, k_offset_std=3.0, zero_q_channel=5, zero_q_tokens=(128, 256),
+                     seed=23), None, False),
+    (inputs.AttnCase("q8_d64_one", 1, 1, 1, 64, seed=25), None, True),
+], ids=lambda x: getattr(x, "name", str(x)))
+def test_prepass_matches_oracle_quantiser(case, N, smooth):
+    _check_prepass(*inputs.attn_inputs(case, N=N), smooth)
+
+
+def _tiny_maxima_inputs(d):
+    """Q block 2 (tokens 256-383) with amax 1e-37, K block 1 (tokens 64-127)
+    with amax 1e-37, V channel 9 of {0, 1e-37} and channel 10 with amax 1e-36:
+    every one of them has a maximum whose inverse overflows fp32."""
+    case = inputs.AttnCase(f"q8tiny{d}", 1, 2, 512, d, seed=24)
+    q, k, v = (inputs.bf16_to_f32(t).copy() for t in inputs.attn_inputs(case))
+    q[:, :, 256:384, :] = 0.0
+    q[:, :, 256:384:2, 3] = 1e-37
+    k[:, :, 64:128, :] = 0.0
+    k[:, :, 64:128:5, 1] = -1e-37
+    v[:, :, :, 9] = 0.0
+    v[:, :, ::3, 9] = 1e-37
+    v[:, :, :, 10] = 0.0
+    v[:, :, 7, 10] = 1e-36
+    return tuple(inputs.bf16_bits(t) for t in (q, k, v))
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_zero_scale_guard_for_maxima_without_a_finite_inverse(d):
+    # An amax so small that 127/amax (or 448/amax) overflows fp32 would give
+    # inv = inf and turn the block's zeros into NaN codes.  The guard treats
+    # such a block or channel as zero: codes and scales equal the oracle's, and
+    # the outputs are finite and meet the 8-bit bar.
+    import diffusion_transformer_attention_attn_b200 as dit
+    q, k, v = _tiny_maxima_inputs(d)
+    _check_prepass(q, k, v, smooth=False)
+    ws = dit.dit_attn_q8_quantize(*_dev(q, k, v), smooth_k=False, pv_mode="fp8")
+    views = dit.q8_views(ws, 1, 2, 512, d, "fp8")
+    assert (views["q_scale"][:, :, 2] == 0).all().item() and (views["k_scale"][:, :, 1] == 0).all().item()
+    assert (views["v_scale"][:, :, 9:11] == 0).all().item()
+    ref = oracle.attention(q, k, v)
+    for mode in ("fp8", "bf16"):
+        for smooth in (False, True):
+            _check(_run(q, k, v, mode, smooth), ref, mode, f"d={d} smooth={smooth}")
 
 
 def test_zero_scale_guard():
@@ -115,6 +160,30 @@ def test_ragged_lengths(N, mode):
     case = inputs.AttnCase(f"q8r{N}", 1, 2, N, 128, k_offset_std=2.0, seed=100 + N)
     q, k, v = inputs.attn_inputs(case)
     _check(_run(q, k, v, mode), oracle.attention(q, k, v), mode, f"N={N}")
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp8"])
+@pytest.mark.parametrize("N", [1, 63, 64, 65, 127, 128, 129, 255, 256, 300, 1000])
+def test_ragged_lengths_d64(N, mode):
+    case = inputs.AttnCase(f"q8r{N}d64", 1, 2, N, 64, k_offset_std=2.0, seed=300 + N)
+    q, k, v = inputs.attn_inputs(case)
+    _check(_run(q, k, v, mode), oracle.attention(q, k, v), mode, f"d=64 N={N}")
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp8"])
+def test_image_shape_d64_sampled_rows(mode):
+    # The 8-bit image recipe (K offsets, a zero Q channel and a zero Q block)
+    # at head dimension 64: B=1, H=24, N=4608.
+    import diffusion_transformer_attention_attn_b200 as dit
+    case = inputs.AttnCase("image_q8_d64", 1, 24, 4608, 64, k_offset_std=5.0, zero_q_channel=7,
+                           zero_q_tokens=(640, 768), seed=26)
+    q, k, v = inputs.attn_inputs(case)
+    o = dit.dit_attn_fwd_q8(*_dev(q, k, v), smooth_k=True, pv_mode=mode)
+    torch.cuda.synchronize()
+    rows = np.union1d(inputs.sample_rows(case.N, 64), [640, 767, 4607])
+    out = from_device_bf16(o[:, :, torch.from_numpy(rows).cuda()])
+    _check(out, oracle.attention(q, k, v, rows=rows), mode, case.name)
+    assert torch.isfinite(o.float()).all().item()
 
 
 @pytest.mark.parametrize("mode", ["bf16", "fp8"])

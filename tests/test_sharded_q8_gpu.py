@@ -1,5 +1,14 @@
 """The token-sharded 8-bit path through the C ABI on one GPU.
 
+Against the oracle: each split entry point on its own —
+dit_attn_q8_channel_stats against oracle.k_channel_sums / channel_amax,
+dit_attn_q8_quantize_global against the oracle's quantisers with the
+combined statistics (both bit for bit), and dit_attn_fwd_q8_prequantized
+against the exact fp64 attention (the 8-bit bar) and against the fp64
+attention over the same codes.
+
+Against the single call:
+
 dit_attn_q8_channel_stats / dit_attn_q8_quantize_global / the codes' move to
 the head-sharded layout / dit_attn_fwd_q8_prequantized must give, bit for
 bit, the codes and the output of the single dit_attn_fwd_q8 call when every
@@ -10,8 +19,9 @@ device copies, as the collectives of a Ulysses group would.
 import numpy as np
 import pytest
 
+import oracle
 from diffusion_transformer_attention_attn_b200 import inputs
-from tests.common import to_device_bf16
+from tests.common import Q8_COSINE, Q8_REL_L1, cosine, from_device_bf16, rel_l1, to_device_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -36,6 +46,85 @@ def _dit():
 def _inputs(N=1024, H=4, seed=2):
     case = inputs.AttnCase("shq8", 1, H, N, 128, k_offset_std=3.0, zero_q_channel=7, seed=seed)
     return [to_device_bf16(x) for x in inputs.attn_inputs(case)]
+
+
+FP8_REL_L1 = 5e-2      # FP8 P·V: e4m3 rounding of V alone costs about 2.7% (see tests/test_q8_gpu.py)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("pv_mode", ["fp8", "bf16"])
+@pytest.mark.parametrize("smooth_k", [True, False])
+def test_split_entry_points_match_the_oracle(d, pv_mode, smooth_k):
+    dit = _dit()
+    world, N, H = 2, 1024, 4
+    case = inputs.AttnCase(f"shq8o{d}", 1, H, N, d, k_offset_std=3.0, zero_q_channel=7, seed=9)
+    q, k, v = inputs.attn_inputs(case)
+    qd, kd, vd = (to_device_bf16(t) for t in (q, k, v))
+    B = 1
+    Nl, hp = N // world, H // world
+    sl = [slice(r * Nl, (r + 1) * Nl) for r in range(world)]
+    fp8 = pv_mode == "fp8"
+    # 1. per-slice statistics against the oracle's sums and maxima
+    stats = [dit.dit_attn_q8_channel_stats(kd[:, :, s], vd[:, :, s], smooth_k=smooth_k, pv_mode=pv_mode) for s in sl]
+    torch.cuda.synchronize()
+    for (ks_dev, va_dev), s in zip(stats, sl):
+        want_sum = oracle.k_channel_sums(k[:, :, s]) if smooth_k else np.zeros((B, H, d))
+        want_max = oracle.channel_amax(v[:, :, s]) if fp8 else np.zeros((B, H, d), dtype=np.float32)
+        np.testing.assert_array_equal(ks_dev.cpu().numpy(), want_sum)
+        np.testing.assert_array_equal(va_dev.cpu().numpy(), want_max)
+    k_sum = sum(x for x, _ in stats)
+    v_amax = torch.stack([y for _, y in stats]).amax(dim=0)
+    # 2. each slice's codes and scales with the combined statistics
+    mean = oracle.mean_from_sums(oracle.k_channel_sums(k), N) if smooth_k else None
+    amax = oracle.channel_amax(v)
+    local = []
+    for s in sl:
+        ws = dit.dit_attn_q8_quantize_global(qd[:, :, s], kd[:, :, s], vd[:, :, s], k_sum, v_amax, N,
+                                             smooth_k=smooth_k, pv_mode=pv_mode)
+        views = dit.q8_views(ws, B, H, Nl, d, pv_mode)
+        local.append(views)
+        got = {n: t.cpu().numpy() for n, t in views.items()}
+        qc, qs = oracle.quant_int8_blocks(q[:, :, s], 128)
+        kc, ks = oracle.quant_int8_blocks(k[:, :, s], 64, mean)
+        np.testing.assert_array_equal(got["q_codes"], qc)
+        np.testing.assert_array_equal(got["q_scale"], qs)
+        np.testing.assert_array_equal(got["k_codes"], kc)
+        np.testing.assert_array_equal(got["k_scale"], ks)
+        if smooth_k:
+            np.testing.assert_array_equal(got["k_mean"], mean)
+        if fp8:
+            vc, vs = oracle.quant_e4m3_with_amax(v[:, :, s], amax)
+            np.testing.assert_array_equal(got["v_codes"], vc)
+            np.testing.assert_array_equal(got["v_scale"], vs)
+    # 3. the attention kernel alone on the gathered head groups
+    out = torch.empty_like(qd)
+    for g in range(world):
+        heads = slice(g * hp, (g + 1) * hp)
+        ws = dit.q8_workspace(B, hp, N, d, pv_mode)
+        dst = dit.q8_views(ws, B, hp, N, d, pv_mode)
+        names = ["q_codes", "k_codes", "q_scale", "k_scale"] + (["v_codes"] if fp8 else [])
+        for n in names:
+            dst[n].copy_(torch.cat([local[r][n][:, heads] for r in range(world)], dim=2))
+        if fp8:
+            dst["v_scale"].copy_(local[0]["v_scale"][:, heads])
+        vh = None if fp8 else vd[:, heads].contiguous()
+        out[:, heads] = dit.dit_attn_fwd_q8_prequantized(ws, B, hp, N, v=vh, pv_mode=pv_mode, d=d)
+    torch.cuda.synchronize()
+    o = from_device_bf16(out)
+    ref = oracle.attention(q, k, v)
+    c, r = cosine(o, ref), rel_l1(o, ref)
+    assert c >= Q8_COSINE and r <= (FP8_REL_L1 if fp8 else Q8_REL_L1), (c, r)
+    # against fp64 attention over the very codes the kernel read (whole sequence)
+    qc, qs = oracle.quant_int8_blocks(q, 128)
+    kc, ks = oracle.quant_int8_blocks(k, 64, mean)
+    if fp8:
+        vc, vs = oracle.quant_e4m3_with_amax(v, amax)
+        emu = oracle.attention_from_codes(qc, qs, kc, ks, vc, vs)
+    else:
+        emu = oracle.attention_from_codes(qc, qs, kc, ks, v)
+    c, r = cosine(o, emu), rel_l1(o, emu)
+    # bf16 P·V: only P's bf16 rounding and fp32 sums remain; FP8 P·V: P's e4m3 rounding too
+    assert c >= 0.9995 and r <= (3.5e-2 if fp8 else 5e-3), (c, r)
 
 
 @pytest.mark.parametrize("pv_mode", ["fp8", "bf16"])
@@ -111,7 +200,7 @@ def test_prequantized_argument_errors():
     o = torch.empty(1, 2, 256, 128, dtype=torch.bfloat16, device="cuda")
     assert lib.dit_attn_fwd_q8_prequantized(ws.data_ptr(), 100, None, o.data_ptr(), 1, 2, 256, 128, None, 0.0, 0,
                                             None) == dit.DIT_ERR_WORKSPACE
-    assert lib.dit_attn_fwd_q8_prequantized(ws.data_ptr(), ws.numel(), None, o.data_ptr(), 1, 2, 256, 64, None, 0.0,
+    assert lib.dit_attn_fwd_q8_prequantized(ws.data_ptr(), ws.numel(), None, o.data_ptr(), 1, 2, 256, 96, None, 0.0,
                                             0, None) == dit.DIT_ERR_UNSUPPORTED
     # bf16-PV mode needs V
     assert lib.dit_attn_fwd_q8_prequantized(ws.data_ptr(), ws.numel(), None, o.data_ptr(), 1, 2, 256, 128, None, 0.0,
