@@ -7,8 +7,6 @@ is no fallback: if the library is missing, importing the binding's entry
 points raises.
 
 Entry points (same names as the C ABI in ``include/dit_attn.h``):
-  * ``attention(q, k, v, backend=None)``           — picks one of the two kernels below by
-    backend name (argument, else DIFFUSION_ATTENTION_BACKEND)
   * ``dit_attn_fwd(q, k, v, o=None, scale=None)``  — bf16 softmax attention
   * ``dit_attn_fwd_ex(q, k, v, ..., lse=...)``      — Nq queries x Nkv keys, optional log-sum-exp
   * ``dit_attn_merge(o_parts, lse_parts)``          — attention over the union of key chunks
@@ -230,32 +228,6 @@ def dit_attn_merge(o_parts, lse_parts, o=None, lse=None, stream=None):
     return o, lse
 
 
-# Backend names of the vLLM-Omni "Diffusion Attention Backends" page, for the
-# two attention kernels of this library.
-ATTENTION_BACKENDS = ("FLASH_ATTN", "SAGE_ATTN")
-
-
-def attention_backend(backend: str | None = None) -> str:
-    """The backend `attention` uses: the argument, else the environment
-    variable DIFFUSION_ATTENTION_BACKEND, else FLASH_ATTN (the page's order of
-    precedence, with this library's bf16 kernel as the platform default)."""
-    name = backend or os.environ.get("DIFFUSION_ATTENTION_BACKEND") or "FLASH_ATTN"
-    name = name.upper()
-    if name not in ATTENTION_BACKENDS:
-        raise ValueError(f"attention backend {name!r}: this library serves {', '.join(ATTENTION_BACKENDS)} "
-                         "(no PyTorch SDPA fallback)")
-    return name
-
-
-def attention(q, k, v, scale: float | None = None, backend: str | None = None, stream=None):
-    """Attention over bf16 [B, H, N, d] CUDA tensors with the selected backend:
-    FLASH_ATTN -> dit_attn_fwd (bf16), SAGE_ATTN -> dit_attn_fwd_q8 (INT8 QKᵀ
-    with K smoothing, FP8 P·V; d = 128).  Returns a new output tensor."""
-    if attention_backend(backend) == "SAGE_ATTN":
-        return dit_attn_fwd_q8(q, k, v, scale=scale, smooth_k=True, pv_mode="fp8", stream=stream)
-    return dit_attn_fwd(q, k, v, scale=scale, stream=stream)
-
-
 def _pv(pv_mode):
     return PV_MODES[pv_mode] if isinstance(pv_mode, str) else int(pv_mode)
 
@@ -318,7 +290,7 @@ def dit_attn_fwd_q8(q, k, v, o=None, scale: float | None = None, smooth_k: bool 
                     workspace=None, stream=None):
     """8-bit attention: INT8 Q (per 128 tokens) and K (per 64 tokens, optional
     channel-mean smoothing), S in int32, P·V in FP8 e4m3 or bf16.  bf16 CUDA
-    tensors [B, H, N, 128].  Returns o."""
+    tensors [B, H, N, d], d = 64 or 128.  Returns o."""
     import torch
     lib = load_library()
     if o is None:

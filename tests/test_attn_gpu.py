@@ -162,14 +162,3 @@ def test_full_size_sampled_rows(case, count):
     assert_bf16_parity(out, ref, case.name)
     # every output finite, and no untouched (garbage) rows
     assert torch.isfinite(od.float()).all().item()
-
-
-def test_backend_names_select_the_kernels(monkeypatch):
-    import diffusion_transformer_attention_attn_b200 as dit
-    q, k, v = (to_device_bf16(t) for t in inputs.attn_inputs(inputs.AttnCase("be", 1, 2, 640, 128, seed=8)))
-    monkeypatch.setenv("DIFFUSION_ATTENTION_BACKEND", "SAGE_ATTN")
-    o8 = dit.attention(q, k, v)
-    o16 = dit.attention(q, k, v, backend="FLASH_ATTN")
-    torch.cuda.synchronize()
-    assert torch.equal(o16, dit.dit_attn_fwd(q, k, v))
-    assert torch.equal(o8, dit.dit_attn_fwd_q8(q, k, v, smooth_k=True, pv_mode="fp8"))
