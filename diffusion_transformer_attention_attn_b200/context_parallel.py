@@ -25,18 +25,51 @@ work), and the cache decision over a sharded residual:
   (``fbc_rel_l1_sums``), one all-reduce adds them, and ``fbc_rel_l1_finish``
   forms rel and the decision on every rank.
 
-The collectives are torch.distributed calls (NCCL between GPUs); the attention,
-the merge and the reductions are the library's kernels.  ``attn_fn``,
-``attn_lse_fn``, ``merge_fn``, ``stats_fn``, ``quant_fn``, ``codes_attn_fn``,
-``sums_fn`` and ``finish_fn`` may be replaced,
-e.g. to run the data movement on CPU ranks.
+The collectives go through a communicator (``TorchComm``: torch.distributed
+calls, NCCL between GPUs); the attention, the merge and the reductions are the
+library's kernels.  ``attn_fn``, ``attn_lse_fn``, ``merge_fn``, ``stats_fn``,
+``quant_fn``, ``codes_attn_fn``, ``sums_fn`` and ``finish_fn`` may be
+replaced, e.g. to run the data movement on CPU ranks, and so may ``comm``,
+any object with the four methods of ``TorchComm``.
 """
 from __future__ import annotations
 
 
-def _group_info(group):
-    import torch.distributed as dist
-    return dist.get_world_size(group), dist.get_rank(group)
+class TorchComm:
+    """The four collective steps the context-parallel schemes take, over a
+    torch.distributed process group (``group`` None: the default group)."""
+
+    def __init__(self, group=None):
+        import torch.distributed as dist
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+
+    def all_to_all(self, recv, send):
+        """Equal split along dim 0: recv[i] = rank i's send[this rank]."""
+        import torch.distributed as dist
+        dist.all_to_all_single(recv, send, group=self.group)
+
+    def all_reduce(self, t, op: str = "sum"):
+        """In place: the elementwise sum ("sum") or maximum ("max") over ranks."""
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.SUM if op == "sum" else dist.ReduceOp.MAX, group=self.group)
+
+    def ring_exchange(self, send, recv):
+        """Start sending ``send`` to rank+1 and receiving rank-1's into
+        ``recv``; returns handles whose ``wait()`` completes the exchange."""
+        import torch.distributed as dist
+        nxt = (self.rank + 1) % self.world
+        prv = (self.rank - 1) % self.world
+        if self.group is not None:
+            nxt = dist.get_global_rank(self.group, nxt)
+            prv = dist.get_global_rank(self.group, prv)
+        ops = [dist.P2POp(dist.isend, send, nxt, self.group), dist.P2POp(dist.irecv, recv, prv, self.group)]
+        return dist.batch_isend_irecv(ops)
+
+
+def _comm(group, comm):
+    return comm if comm is not None else TorchComm(group)
 
 
 def _default_attn(q, k, v):
@@ -54,7 +87,7 @@ def _default_merge(outs, lses):
     return dit_attn_merge(outs, lses, lse=True)
 
 
-def seq_to_heads(xs, world: int, group=None):
+def seq_to_heads(xs, world: int, group=None, comm=None):
     """All-to-all of sequence-sharded tensors to head-sharded ones.
 
     xs: list of [B, H, Nl, d] tensors (this rank's Nl = N/P tokens, all heads),
@@ -63,37 +96,36 @@ def seq_to_heads(xs, world: int, group=None):
     travel in one all-to-all.
     """
     import torch
-    import torch.distributed as dist
     B, H, Nl, d = xs[0].shape
     P = world
     hp = H // P
     # [P (destination head group), T, B, H/P, Nl, d]
     send = torch.stack([x.reshape(B, P, hp, Nl, d) for x in xs], dim=0).permute(2, 0, 1, 3, 4, 5).contiguous()
     recv = torch.empty_like(send)
-    dist.all_to_all_single(recv, send, group=group)
+    _comm(group, comm).all_to_all(recv, send)
     # recv[src] = src's tokens of my heads -> [T, B, H/P, P*Nl, d]
     out = recv.permute(1, 2, 3, 0, 4, 5).reshape(len(xs), B, hp, P * Nl, d)
     return [out[i] for i in range(len(xs))]
 
 
-def heads_to_seq(y, world: int, group=None):
+def heads_to_seq(y, world: int, group=None, comm=None):
     """Inverse of ``seq_to_heads`` for one tensor: [B, H/P, P*Nl, d] ->
     [B, H, Nl, d] (this rank's tokens, all heads, head groups rank-major)."""
     import torch
-    import torch.distributed as dist
     B, hp, N, d = y.shape
     P = world
     Nl = N // P
     send = y.reshape(B, hp, P, Nl, d).permute(2, 0, 1, 3, 4).contiguous()   # [P (token owner), B, H/P, Nl, d]
     recv = torch.empty_like(send)
-    dist.all_to_all_single(recv, send, group=group)
+    _comm(group, comm).all_to_all(recv, send)
     return recv.permute(1, 0, 2, 3, 4).reshape(B, P * hp, Nl, d)
 
 
-def ulysses_attention(q, k, v, group=None, attn_fn=None):
+def ulysses_attention(q, k, v, group=None, attn_fn=None, comm=None):
     """Attention over the full sequence from sequence-sharded [B, H, N/P, d]
     q, k, v; returns this rank's [B, H, N/P, d] output."""
-    world, _ = _group_info(group)
+    comm = _comm(group, comm)
+    world = comm.world
     B, H, Nl, d = q.shape
     if H % world:
         raise ValueError(f"{H} heads do not split over {world} ranks")
@@ -102,31 +134,26 @@ def ulysses_attention(q, k, v, group=None, attn_fn=None):
     attn = attn_fn or _default_attn
     if world == 1:
         return attn(q, k, v)
-    qh, kh, vh = seq_to_heads([q, k, v], world, group)
-    return heads_to_seq(attn(qh, kh, vh), world, group)
+    qh, kh, vh = seq_to_heads([q, k, v], world, comm=comm)
+    return heads_to_seq(attn(qh, kh, vh), world, comm=comm)
 
 
-def ring_attention(q, k, v, group=None, attn_lse_fn=None, merge_fn=None):
+def ring_attention(q, k, v, group=None, attn_lse_fn=None, merge_fn=None, comm=None):
     """Attention of this rank's queries [B, H, Nl, d] to all ranks' keys, the
     K/V chunks travelling around the ring (rank r sends to r+1 and receives
     from r-1).  Returns (o, lse) for the local queries."""
     import torch
-    import torch.distributed as dist
-    world, rank = _group_info(group)
+    comm = _comm(group, comm)
+    world = comm.world
     attn = attn_lse_fn or _default_attn_lse
     merge = merge_fn or _default_merge
     kv = torch.stack([k, v], dim=0).contiguous()
     outs, lses = [], []
-    nxt = (rank + 1) % world
-    prv = (rank - 1) % world
     for step in range(world):
         reqs = []
         if step + 1 < world:
             buf = torch.empty_like(kv)
-            g_nxt = dist.get_global_rank(group, nxt) if group is not None else nxt
-            g_prv = dist.get_global_rank(group, prv) if group is not None else prv
-            ops = [dist.P2POp(dist.isend, kv, g_nxt, group), dist.P2POp(dist.irecv, buf, g_prv, group)]
-            reqs = dist.batch_isend_irecv(ops)
+            reqs = comm.ring_exchange(kv, buf)
         o_c, l_c = attn(q, kv[0], kv[1])
         outs.append(o_c)
         lses.append(l_c)
@@ -153,14 +180,13 @@ def _default_finish(sums, threshold):
     return fbc_rel_l1_finish(sums, threshold)
 
 
-def sharded_fbc_rel_l1(r_cur, r_prev, threshold: float, group=None, sums_fn=None, finish_fn=None):
+def sharded_fbc_rel_l1(r_cur, r_prev, threshold: float, group=None, sums_fn=None, finish_fn=None, comm=None):
     """(rel, skip) of a residual whose elements are split across the ranks of
     ``group``; every rank gets the same result."""
-    import torch.distributed as dist
     sums = (sums_fn or _default_sums)(r_cur, r_prev)
-    world, _ = _group_info(group)
-    if world > 1:
-        dist.all_reduce(sums, op=dist.ReduceOp.SUM, group=group)
+    comm = _comm(group, comm)
+    if comm.world > 1:
+        comm.all_reduce(sums, "sum")
     return (finish_fn or _default_finish)(sums, threshold)
 
 
@@ -193,14 +219,14 @@ def _default_codes_attn(parts, v, pv_mode):
 
 
 def ulysses_attention_q8(q, k, v, group=None, smooth_k: bool = True, pv_mode="fp8", stats_fn=None, quant_fn=None,
-                         codes_attn_fn=None):
+                         codes_attn_fn=None, comm=None):
     """8-bit attention over the full sequence from sequence-sharded
     [B, H, N/P, d] q, k, v, with the all-to-all carrying the 8-bit codes
     (bf16 V instead in bf16-PV mode).  N/P must be a multiple of 128 (whole
     Q blocks per rank).  Returns this rank's [B, H, N/P, d] output."""
     import torch
-    import torch.distributed as dist
-    world, rank = _group_info(group)
+    comm = _comm(group, comm)
+    world, rank = comm.world, comm.rank
     B, H, Nl, d = q.shape
     if H % world:
         raise ValueError(f"{H} heads do not split over {world} ranks")
@@ -209,24 +235,24 @@ def ulysses_attention_q8(q, k, v, group=None, smooth_k: bool = True, pv_mode="fp
     fp8 = pv_mode in ("fp8", 0)
     k_sum, v_amax = (stats_fn or _default_stats)(k, v, smooth_k, pv_mode)
     if world > 1:
-        dist.all_reduce(k_sum, op=dist.ReduceOp.SUM, group=group)
-        dist.all_reduce(v_amax, op=dist.ReduceOp.MAX, group=group)
+        comm.all_reduce(k_sum, "sum")
+        comm.all_reduce(v_amax, "max")
     local = (quant_fn or _default_quant)(q, k, v, k_sum, v_amax, Nl * world, smooth_k, pv_mode)
     hp = H // world
     names = [n for n in CODE_KEYS if n in local]
     parts = {}
     if world > 1:
         # 1-byte codes travel as 32-bit words (d is a multiple of 4).
-        moved = seq_to_heads([local[n].contiguous().view(torch.int32) for n in names], world, group)
+        moved = seq_to_heads([local[n].contiguous().view(torch.int32) for n in names], world, comm=comm)
         for n, t in zip(names, moved):
             parts[n] = t.contiguous().view(local[n].dtype)
         for n in ("q_scale", "k_scale"):
-            parts[n] = seq_to_heads([local[n].unsqueeze(-1)], world, group)[0].squeeze(-1).contiguous()
-        vh = None if fp8 else seq_to_heads([v], world, group)[0].contiguous()
+            parts[n] = seq_to_heads([local[n].unsqueeze(-1)], world, comm=comm)[0].squeeze(-1).contiguous()
+        vh = None if fp8 else seq_to_heads([v], world, comm=comm)[0].contiguous()
     else:
         parts = {n: local[n] for n in names + ["q_scale", "k_scale"]}
         vh = None if fp8 else v
     if fp8:
         parts["v_scale"] = local["v_scale"][:, rank * hp:(rank + 1) * hp].contiguous()
     oh = (codes_attn_fn or _default_codes_attn)(parts, vh, pv_mode)
-    return oh if world == 1 else heads_to_seq(oh, world, group)
+    return oh if world == 1 else heads_to_seq(oh, world, comm=comm)

@@ -5,8 +5,9 @@ Some callers hold only their input and output pointers, for example a plugin
 inside an inference engine, or a module whose framework's caching allocator
 owns all device memory.  They cannot pass fbc_rel_l1 a workspace.  The
 no-alloc variant keeps its scratch in a fixed array inside the library.  Its
-result must match the workspace entry point on the same inputs, and stay
-correct from one call to the next, since every call shares that array.
+result must match the fp64 oracle and the workspace entry point on the same
+inputs, and stay correct from one call to the next, since every call shares
+that array.
 
 This file is collected last on purpose.  If it fails, a run that stops at the
 first failure has already run every other test.
@@ -16,6 +17,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 from diffusion_transformer_attention_attn_b200 import inputs
 from tests.common import FBC_REL_ERR
 
@@ -72,11 +74,14 @@ def test_no_alloc_matches_workspace_entry_point_on_consecutive_calls(lib):
         dc, dp = _dev(cur.reshape(-1)), _dev(prev.reshape(-1))
         n = cur.size
         ref_rel, ref_skip = _with_workspace(lib, dc, dp, n, dtype, thr, stream)
+        o_rel, o_skip = oracle.fbc_rel_l1(cur, prev, thr)
         # two calls in a row through the shared scratch array
         for _ in range(2):
             rel, skip = _no_alloc(lib, dc, dp, n, dtype, thr, stream)
             torch.cuda.synchronize()
             r, rr = rel.item(), ref_rel.item()
+            assert abs(r - o_rel) <= FBC_REL_ERR * abs(o_rel), (case.name, r, o_rel)
+            assert int(skip.item()) == o_skip, case.name
             assert abs(r - rr) <= FBC_REL_ERR * abs(rr), (case.name, r, rr)
             assert int(skip.item()) == int(ref_skip.item()), case.name
     import diffusion_transformer_attention_attn_b200 as dit
