@@ -566,15 +566,30 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     prepass_ms = ep[0].elapsed_time(ep[1]) / K
 
+    # ---- the 8-bit call with bf16 P·V (informational, outside the timed step):
+    # the mode that meets the 8-bit tolerance in both cosine and relative L1
+    qws16 = dit.q8_workspace(case.B, case.H, case.N, case.d, "bf16", dev)
+
+    def q8_bf16pv():
+        dit.dit_attn_fwd_q8(dq, dk, dv, o=do8, smooth_k=True, pv_mode="bf16", workspace=qws16)
+
+    q8_bf16pv()
+    torch.cuda.synchronize(dev)
+    q8b_ms = _time_calls(torch, stream, q8_bf16pv, K)
+    q8(do8)   # leave the FP8-PV output in do8 for the comparison timings below
+    torch.cuda.synchronize(dev)
+    del qws16
+
     # ---- the step caches and the output comparison (outside the timed step)
     extra = {} if args.no_next_rows else measure_next_rows(dit, torch, dev, stream, dcur, dprev, do, do8, dq, dk,
                                                                  dv, case, K)
 
     # ---- max over ranks
     keys = sorted(extra)
-    vals = max_over_ranks([ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms] + [extra[k] for k in keys], dev, ws)
-    ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms = vals[:6]
-    extra = dict(zip(keys, vals[6:]))
+    vals = max_over_ranks([ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms, q8b_ms] + [extra[k] for k in keys], dev,
+                          ws)
+    ms, e2e_ms, attn_ms, q8_ms, fbc_ms, prepass_ms, q8b_ms = vals[:7]
+    extra = dict(zip(keys, vals[7:]))
 
     flops = 4.0 * case.B * case.H * case.N * case.N * case.d  # one attention call
     value = ws * K * 2 * flops / (ms * 1e-3) / 1e12
@@ -601,10 +616,18 @@ def run_ours(args):
                     "q8_call_ms": q8_ms, "q8_call_tflops": q8_tflops, "q8_prepass_ms": prepass_ms,
                     "q8_attn_tflops": q8_attn_tflops, "q8_attn_frac_of_fp8_peak": q8_attn_tflops / peak8,
                     "q8_speedup_vs_bf16": attn_ms / q8_ms,
+                    "q8_bf16pv_call_ms": q8b_ms, "q8_bf16pv_call_tflops": flops / (q8b_ms * 1e-3) / 1e12,
+                    "q8_bf16pv_speedup_vs_bf16": attn_ms / q8b_ms,
                     "fbc_ms": fbc_ms, "fbc_gbs": fbc_gbs,
                     "fbc_frac_of_measured_hbm": fbc_gbs / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
                     "fbc_frac_of_spec_8000": fbc_gbs / SPEC_HBM_GBS},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "parity": {
+            "bf16": "max|dO| <= 2e-2 and rel-L1 <= 5e-3 against the fp64 oracle: met",
+            "q8_fp8_pv": "the step's 8-bit call. cosine >= 0.999: met; rel-L1 <= 2e-2: NOT met (tested at "
+                         "5e-2; e4m3 rounding of V alone costs about 2.7% rel-L1 on N(0,1) inputs)",
+            "q8_bf16_pv": "kernels.q8_bf16pv_*: cosine >= 0.999 and rel-L1 <= 2e-2: met",
+            "fbc": "relative error <= 1e-5 and identical decisions: met"},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
         "next_rows": None if args.no_next_rows else next_rows_report(extra, fcase, case, peaks),
