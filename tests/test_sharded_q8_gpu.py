@@ -57,7 +57,9 @@ FP8_REL_L1 = 5e-2      # FP8 P·V: e4m3 rounding of V alone costs about 2.7% (se
 def test_split_entry_points_match_the_oracle(d, pv_mode, smooth_k):
     dit = _dit()
     world, N, H = 2, 1024, 4
-    case = inputs.AttnCase(f"shq8o{d}", 1, H, N, d, k_offset_std=3.0, zero_q_channel=7, seed=9)
+    # K's per-channel offsets need the smoothing to meet the 8-bit bar (without
+    # it they set the INT8 scale); the unsmoothed runs take plain N(0,1) keys.
+    case = inputs.AttnCase(f"shq8o{d}", 1, H, N, d, k_offset_std=3.0 if smooth_k else 0.0, zero_q_channel=7, seed=9)
     q, k, v = inputs.attn_inputs(case)
     qd, kd, vd = (to_device_bf16(t) for t in (q, k, v))
     B = 1
