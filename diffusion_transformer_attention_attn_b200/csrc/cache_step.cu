@@ -47,6 +47,7 @@ __device__ __forceinline__ void record(dit_cache_trace* trace, int32_t cap, int 
 }
 
 struct EpiFbcPolicy {
+    static constexpr bool kProgrammatic = false;  // reads the state the previous step wrote first
     int32_t warmup, max_cached, max_cont;
     float threshold;
     dit_cache_state* st;
@@ -92,6 +93,7 @@ struct EpiFbcPolicy {
 };
 
 struct EpiTeaCache {
+    static constexpr bool kProgrammatic = false;
     double coeffs[kMaxCoeffs];
     int32_t n_coeffs;
     float threshold;

@@ -6,7 +6,9 @@
 // reused.
 //
 // One HBM-bound launch of the shared relative-L1 reduction (rel_l1_reduce.cuh)
-// whose epilogue writes rel and skip.
+// whose epilogue writes rel and skip, launched so that it overlaps the tail of
+// the kernel before it (programmatic launch with an L2 prefetch of its first
+// loads).
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -20,6 +22,7 @@ namespace ditk {
 namespace {
 
 struct EpiThreshold {
+    static constexpr bool kProgrammatic = true;
     float threshold;
     double* out_rel;
     int32_t* out_skip;
@@ -33,6 +36,7 @@ struct EpiThreshold {
 
 // The two sums themselves (for a residual sharded across devices).
 struct EpiSums {
+    static constexpr bool kProgrammatic = true;
     double* out;
     __device__ bool evaluate() const { return true; }
     __device__ void finish(double num, double den, bool) const {

@@ -21,6 +21,16 @@
 // TeaCache accumulator needs on every step.  An epilogue may declare that the
 // sums are not needed (evaluate() false): the kernel then reads nothing and
 // only runs the epilogue.
+//
+// An epilogue with kProgrammatic = true (the plain decision and the sums,
+// whose kernels always read their inputs) is launched as a programmatic
+// dependent of the kernel before it in the stream: its blocks may become
+// resident while that kernel finishes.  Each block then asks L2 for its first
+// trip of both inputs (cp.async.bulk.prefetch.L2, a hint) and waits
+// (griddepcontrol.wait) for the preceding grid and its memory before any load,
+// so the DRAM latency of the first loads overlaps the previous kernel's tail.
+// The loads themselves come after the wait and read coherent L2, so inputs
+// that the previous kernel writes are seen as written.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -92,6 +102,22 @@ __global__ void __launch_bounds__(kFbcThreads)
                   void* prev_tail, int tail, Epi epi, FbcWs* ws) {
     __shared__ double2 sh[kFbcThreads / 32];
     __shared__ bool is_last;
+    if constexpr (Epi::kProgrammatic) {
+        // Threads 0 .. 2·kFbcUnroll−1: one contiguous run of this block's
+        // first trip each (trip u, input cur or prev).
+        if (threadIdx.x < 2 * kFbcUnroll) {
+            const int64_t u = threadIdx.x >> 1;
+            const int64_t v0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + u * gridDim.x * blockDim.x;
+            if (v0 < nvec) {
+                const int64_t nv = min(static_cast<int64_t>(blockDim.x), nvec - v0);
+                const VecT* base = (threadIdx.x & 1) ? static_cast<const VecT*>(prev) : cur;
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + v0),
+                             "r"(static_cast<uint32_t>(nv * sizeof(VecT)))
+                             : "memory");
+            }
+        }
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
     double2* partials = reinterpret_cast<double2*>(ws + 1);
     const bool eval = epi.evaluate();
 
@@ -143,16 +169,20 @@ __global__ void __launch_bounds__(kFbcThreads)
             }
         }
     }
+    // This block has loaded all it reads: a programmatic dependent of this
+    // grid may be scheduled (no effect when there is none).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     rl1_block_sum2(num, den, sh);
     if (threadIdx.x == 0) {
         partials[blockIdx.x] = make_double2(num, den);
-        __threadfence();
-        const unsigned int t = atomicAdd(&ws->ticket, 1u);
+        // Release publishes this block's partial; the last block's acquire
+        // (with the barrier below) makes every partial visible to its threads.
+        unsigned int t;
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(t) : "l"(&ws->ticket) : "memory");
         is_last = (t == gridDim.x - 1);
     }
     __syncthreads();
     if (!is_last) return;
-    __threadfence();
     // Last block: fixed-order sum of the partials.
     double a = 0.0, b = 0.0;
     for (int k = threadIdx.x; k < static_cast<int>(gridDim.x); k += blockDim.x) {
@@ -197,30 +227,40 @@ inline int rel_l1_blocks(int64_t nvec) {
 }
 
 // Launch over n elements of dtype 0 (fp32) or 1 (bf16).  prev must be
-// writable when kCopy.
+// writable when kCopy.  Epi::kProgrammatic selects the programmatic
+// (overlapped) launch described at the top of this file.
 template <bool kCopy, typename Epi>
 cudaError_t launch_rel_l1(const void* cur, const void* prev, int64_t n, int dtype, const Epi& epi, void* workspace,
                           cudaStream_t stream) {
     FbcWs* ws = static_cast<FbcWs*>(workspace);
     void* pv = const_cast<void*>(prev);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kFbcThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = Epi::kProgrammatic ? 1 : 0;
     if (dtype == 0) {
         const int64_t nvec = n / 4;
         const int tail = static_cast<int>(n - nvec * 4);
         const float* c = static_cast<const float*>(cur);
         float* p = static_cast<float*>(pv);
-        rel_l1_kernel<float4, 4, kCopy, Epi><<<rel_l1_blocks(nvec), kFbcThreads, 0, stream>>>(
-            reinterpret_cast<const float4*>(c), reinterpret_cast<float4*>(p), nvec, c + nvec * 4, p + nvec * 4,
-            tail, epi, ws);
-    } else {
-        const int64_t nvec = n / 8;
-        const int tail = static_cast<int>(n - nvec * 8);
-        const __nv_bfloat16* c = static_cast<const __nv_bfloat16*>(cur);
-        __nv_bfloat16* p = static_cast<__nv_bfloat16*>(pv);
-        rel_l1_kernel<uint4, 8, kCopy, Epi><<<rel_l1_blocks(nvec), kFbcThreads, 0, stream>>>(
-            reinterpret_cast<const uint4*>(c), reinterpret_cast<uint4*>(p), nvec, c + nvec * 8, p + nvec * 8, tail,
-            epi, ws);
+        cfg.gridDim = dim3(rel_l1_blocks(nvec));
+        return cudaLaunchKernelEx(&cfg, rel_l1_kernel<float4, 4, kCopy, Epi>, reinterpret_cast<const float4*>(c),
+                                  reinterpret_cast<float4*>(p), nvec, static_cast<const void*>(c + nvec * 4),
+                                  static_cast<void*>(p + nvec * 4), tail, epi, ws);
     }
-    return cudaGetLastError();
+    const int64_t nvec = n / 8;
+    const int tail = static_cast<int>(n - nvec * 8);
+    const __nv_bfloat16* c = static_cast<const __nv_bfloat16*>(cur);
+    __nv_bfloat16* p = static_cast<__nv_bfloat16*>(pv);
+    cfg.gridDim = dim3(rel_l1_blocks(nvec));
+    return cudaLaunchKernelEx(&cfg, rel_l1_kernel<uint4, 8, kCopy, Epi>, reinterpret_cast<const uint4*>(c),
+                              reinterpret_cast<uint4*>(p), nvec, static_cast<const void*>(c + nvec * 8),
+                              static_cast<void*>(p + nvec * 8), tail, epi, ws);
 }
 
 }  // namespace ditk
