@@ -68,7 +68,9 @@ struct Q8Cfg {
     static constexpr uint32_t kIdescPV = FP8 ? make_idesc(1, 0, 0, 0, 1, 128, D) : make_idesc(1, 1, 1, 0, 1, 128, D);
     static constexpr float kShift = FP8 ? 6.5f : 0.0f;     // log2 of P's scale
     static constexpr float kThresh = FP8 ? 2.0f : 8.0f;    // rescale threshold (log2)
-    static constexpr int kEmuOf8 = FP8 ? 2 : 1;            // exp2 pairs (of 8) on the FMA pipe (tuned)
+    // exp2 pairs (of 8) on the FMA pipe (tuned): FP8 P takes the quadratic
+    // (exp2_poly2q, 3 pairs in 8), bf16 P the cubic (1 in 8).
+    static constexpr int kEmuOf8 = FP8 ? 3 : 1;
 };
 
 struct Bars {
@@ -382,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              __int_as_float(static_cast<int>(r[(i + 1) >> 5][(i + 1) & 31]) + 0x4B400000));
                 const float2 t = __ffma2_rn(f, cc, nb);
                 if (((i >> 1) & 7) < C::kEmuOf8) {
-                    const float2 e = exp2_poly2(t);
+                    const float2 e = FP8 ? exp2_poly2q(t) : exp2_poly2(t);
                     p[i] = e.x;
                     p[i + 1] = e.y;
                 } else {

@@ -313,6 +313,21 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                        __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
+// The same with a quadratic for 2^r (relative-error minimax on [-1/2, 1/2],
+// fitted for this library, max relative error 1.73e-3): one FFMA2 fewer per
+// pair, for P stored as e4m3, whose own rounding step is 2^-4 relative.
+__device__ __forceinline__ float2 exp2_poly2q(float2 x) {
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+    const float2 jf = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 r = __ffma2_rn(jf, make_float2(-1.f, -1.f), x);
+    float2 p = __ffma2_rn(make_float2(0.2384289674f, 0.2384289674f), r, make_float2(0.7034480172f, 0.7034480172f));
+    p = __ffma2_rn(p, r, make_float2(1.0004431359f, 1.0004431359f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` goes to bits 0-15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
