@@ -63,6 +63,8 @@ SIGNATURES = {
     "dit_attn_q8_channel_stats": (_i, [_p, _p, _i, _i, _i, _i, _p, _i, _i, _p, _p, _p, _sz, _p]),
     "dit_attn_q8_quantize_global": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _i, _i, _p, _p, _i64, _p, _sz, _p]),
     "dit_attn_fwd_q8_prequantized": (_i, [_p, _sz, _p, _p, _i, _i, _i, _i, _p, _f, _i, _p]),
+    "dit_attn_q8_quantize_scatter": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _i, _i, _p, _p, _i, _i, _p, _sz, _p, _sz,
+                                          _p]),
     "fbc_rel_l1_workspace_bytes": (_sz, [_i64]),
     "fbc_rel_l1": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p, _sz, _p]),
     "fbc_rel_l1_noalloc": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p]),
@@ -355,6 +357,28 @@ def dit_attn_q8_quantize_global(q, k, v, k_sum, v_amax, n_total: int, smooth_k: 
                                          int(bool(smooth_k)), _pv(pv_mode), k_sum.data_ptr(), v_amax.data_ptr(),
                                          int(n_total), workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
     _check(st, "dit_attn_q8_quantize_global")
+    return workspace
+
+
+def dit_attn_q8_quantize_scatter(q, k, v, k_sum, v_amax, rank: int, world: int, dst_workspaces, dst_workspace_bytes,
+                                 smooth_k: bool = True, pv_mode="fp8", workspace=None, stream=None):
+    """Quantise this rank's token slice with the combined statistics and store
+    its codes and block scales straight into the head-sharded workspaces of
+    the group's ranks (``dst_workspaces``: ``world`` device addresses, ints;
+    peer-mapped on a multi-GPU node).  The caller completes every rank's
+    stores before running dit_attn_fwd_q8_prequantized.  Returns the slice
+    workspace (K mean, V scales)."""
+    lib = load_library()
+    _check_attn_tensors(q, k, v, None)
+    B, H, N, d = q.shape
+    if workspace is None:
+        workspace = q8_workspace(B, H, N, d, pv_mode, q.device)
+    ptrs = (ctypes.c_void_p * len(dst_workspaces))(*[int(x) for x in dst_workspaces])
+    st = lib.dit_attn_q8_quantize_scatter(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, _attn_strides(q),
+                                          int(bool(smooth_k)), _pv(pv_mode), k_sum.data_ptr(), v_amax.data_ptr(),
+                                          int(rank), int(world), ptrs, int(dst_workspace_bytes),
+                                          workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(st, "dit_attn_q8_quantize_scatter")
     return workspace
 
 

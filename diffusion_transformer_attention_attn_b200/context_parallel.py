@@ -19,7 +19,10 @@ work), and the cache decision over a sharded residual:
   V maxima (``dit_attn_q8_channel_stats``), two all-reduces combine them, each
   rank quantises its own tokens (``dit_attn_q8_quantize_global``), the codes
   and block scales travel to the head-sharded layout, and the attention runs
-  on them (``dit_attn_fwd_q8_prequantized``).
+  on them (``dit_attn_fwd_q8_prequantized``).  With ``fused=True`` the
+  quantisers store the codes straight into every rank's head-sharded
+  workspace (``dit_attn_q8_quantize_scatter``, peer memory between GPUs), so
+  the all-to-all of the codes is no separate step.
 * ``sharded_fbc_rel_l1`` — the first-block-cache difference of a residual
   sharded like the sequence: each rank reduces its slice to two sums
   (``fbc_rel_l1_sums``), one all-reduce adds them, and ``fbc_rel_l1_finish``
@@ -30,7 +33,8 @@ calls, NCCL between GPUs); the attention, the merge and the reductions are the
 library's kernels.  ``attn_fn``, ``attn_lse_fn``, ``merge_fn``, ``stats_fn``,
 ``quant_fn``, ``codes_attn_fn``, ``sums_fn`` and ``finish_fn`` may be
 replaced, e.g. to run the data movement on CPU ranks, and so may ``comm``,
-any object with the four methods of ``TorchComm``.
+any object with the methods of ``TorchComm`` (the fused 8-bit path also uses
+``shared_workspace`` and ``barrier``).
 """
 from __future__ import annotations
 
@@ -44,6 +48,7 @@ class TorchComm:
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
+        self._shared = {}
 
     def all_to_all(self, recv, send):
         """Equal split along dim 0: recv[i] = rank i's send[this rank]."""
@@ -66,6 +71,29 @@ class TorchComm:
             prv = dist.get_global_rank(self.group, prv)
         ops = [dist.P2POp(dist.isend, send, nxt, self.group), dist.P2POp(dist.irecv, recv, prv, self.group)]
         return dist.batch_isend_irecv(ops)
+
+    def shared_workspace(self, nbytes: int, device):
+        """A device buffer of ``nbytes`` on every rank, mapped into every
+        rank's address space (torch symmetric memory over NVLink): returns
+        (this rank's buffer, every rank's device address).  The buffer of a
+        given size is made once and reused.  Not run on more than one GPU
+        here."""
+        import torch
+        import torch.distributed as dist
+        import torch.distributed._symmetric_memory as symm
+        key = (int(nbytes), str(device))
+        if key not in self._shared:
+            buf = symm.empty(nbytes, dtype=torch.uint8, device=device)
+            handle = symm.rendezvous(buf, self.group if self.group is not None else dist.group.WORLD)
+            self._shared[key] = (buf, [int(p) for p in handle.buffer_ptrs])
+        return self._shared[key]
+
+    def barrier(self):
+        """Every rank's work issued so far on the current stream has completed."""
+        import torch
+        import torch.distributed as dist
+        torch.cuda.current_stream().synchronize()
+        dist.barrier(group=self.group)
 
 
 def _comm(group, comm):
@@ -219,14 +247,18 @@ def _default_codes_attn(parts, v, pv_mode):
 
 
 def ulysses_attention_q8(q, k, v, group=None, smooth_k: bool = True, pv_mode="fp8", stats_fn=None, quant_fn=None,
-                         codes_attn_fn=None, comm=None):
+                         codes_attn_fn=None, comm=None, fused: bool = False):
     """8-bit attention over the full sequence from sequence-sharded
     [B, H, N/P, d] q, k, v, with the all-to-all carrying the 8-bit codes
     (bf16 V instead in bf16-PV mode).  N/P must be a multiple of 128 (whole
-    Q blocks per rank).  Returns this rank's [B, H, N/P, d] output."""
+    Q blocks per rank).  With ``fused`` the quantisers scatter the codes into
+    every rank's workspace directly (the communicator supplies the shared
+    workspaces).  Returns this rank's [B, H, N/P, d] output."""
     import torch
     comm = _comm(group, comm)
     world, rank = comm.world, comm.rank
+    if fused and world > 1:
+        return _ulysses_q8_fused(q, k, v, comm, smooth_k, pv_mode, stats_fn)
     B, H, Nl, d = q.shape
     if H % world:
         raise ValueError(f"{H} heads do not split over {world} ranks")
@@ -256,3 +288,30 @@ def ulysses_attention_q8(q, k, v, group=None, smooth_k: bool = True, pv_mode="fp
         parts["v_scale"] = local["v_scale"][:, rank * hp:(rank + 1) * hp].contiguous()
     oh = (codes_attn_fn or _default_codes_attn)(parts, vh, pv_mode)
     return oh if world == 1 else heads_to_seq(oh, world, comm=comm)
+
+
+def _ulysses_q8_fused(q, k, v, comm, smooth_k, pv_mode, stats_fn):
+    """``ulysses_attention_q8`` with the code all-to-all fused into the
+    quantisers (dit_attn_q8_quantize_scatter)."""
+    from . import dit_attn_fwd_q8_prequantized, dit_attn_q8_quantize_scatter, dit_attn_q8_workspace_bytes
+    world, rank = comm.world, comm.rank
+    B, H, Nl, d = q.shape
+    if H % world:
+        raise ValueError(f"{H} heads do not split over {world} ranks")
+    if Nl % 128:
+        raise ValueError("each rank must hold whole 128-token blocks")
+    fp8 = pv_mode in ("fp8", 0)
+    hp, N = H // world, Nl * world
+    k_sum, v_amax = (stats_fn or _default_stats)(k, v, smooth_k, pv_mode)
+    comm.all_reduce(k_sum, "sum")
+    comm.all_reduce(v_amax, "max")
+    nbytes = dit_attn_q8_workspace_bytes(B, hp, N, d, pv_mode)
+    ws_dst, ptrs = comm.shared_workspace(nbytes, q.device)
+    dit_attn_q8_quantize_scatter(q, k, v, k_sum, v_amax, rank, world, ptrs, nbytes, smooth_k=smooth_k,
+                                 pv_mode=pv_mode)
+    vh = None if fp8 else seq_to_heads([v], world, comm=comm)[0].contiguous()
+    comm.barrier()          # every rank's codes have landed in every workspace
+    oh = dit_attn_fwd_q8_prequantized(ws_dst, B, hp, N, v=vh, pv_mode=pv_mode, d=d)
+    out = heads_to_seq(oh, world, comm=comm)
+    comm.barrier()          # no rank reuses its workspace before the others finished reading theirs
+    return out

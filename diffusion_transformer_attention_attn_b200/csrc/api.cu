@@ -368,6 +368,46 @@ dit_status dit_attn_q8_quantize_global(const void* q, const void* k, const void*
     return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
+dit_status dit_attn_q8_quantize_scatter(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                                        const int64_t* strides, int smooth_k, int pv_mode, const double* k_sum,
+                                        const float* v_amax, int rank, int world, void* const* dst_workspaces,
+                                        size_t dst_workspace_bytes, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+    int64_t sb, sh, sn;
+    dit_status st = check_attn_args(q, k, v, nullptr, B, H, N, d, strides, &sb, &sh, &sn, false);
+    if (st != DIT_OK) return st;
+    if ((st = check_q8_args(d, smooth_k, pv_mode, workspace, workspace_bytes, B, H, N)) != DIT_OK) return st;
+    if (world < 1 || world > kQ8MaxRanks || rank < 0 || rank >= world) return DIT_ERR_INVALID_ARG;
+    if (H % world != 0 || (world > 1 && N % 128 != 0)) return DIT_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(N) * world > (int64_t(1) << 30)) return DIT_ERR_UNSUPPORTED;
+    if (!k_sum || !v_amax || (reinterpret_cast<uintptr_t>(k_sum) & 7u) || (reinterpret_cast<uintptr_t>(v_amax) & 3u))
+        return DIT_ERR_INVALID_ARG;
+    if (!dst_workspaces) return DIT_ERR_INVALID_ARG;
+    const int pv_fp8 = pv_mode == DIT_PV_FP8_E4M3;
+    const size_t need = q8_layout(B, H / world, N * world, d, pv_fp8).total;
+    if (dst_workspace_bytes < need) return DIT_ERR_WORKSPACE;
+    const int64_t local = static_cast<int64_t>(q8_layout(B, H, N, d, pv_fp8).total);
+    const int64_t span = ((B - 1) * sb + (H - 1) * sh + (N - 1) * sn + d) * 2;
+    uint8_t* dst[kQ8MaxRanks];
+    for (int r = 0; r < world; ++r) {
+        dst[r] = static_cast<uint8_t*>(dst_workspaces[r]);
+        if (!dst[r] || (reinterpret_cast<uintptr_t>(dst[r]) & 255u) != 0) return DIT_ERR_WORKSPACE;
+        // every destination is distinct from the others, the slice workspace and the inputs
+        if (overlap_bytes(dst[r], static_cast<int64_t>(need), workspace, local)) return DIT_ERR_WORKSPACE;
+        for (const void* t : {q, k, v})
+            if (overlap_bytes(dst[r], static_cast<int64_t>(need), t, span)) return DIT_ERR_WORKSPACE;
+        for (int u = 0; u < r; ++u)
+            if (overlap_bytes(dst[r], static_cast<int64_t>(need), dst[u], static_cast<int64_t>(need)))
+                return DIT_ERR_WORKSPACE;
+    }
+    DeviceState* ds = device_state(&st);
+    if (!ds) return st;
+    cudaError_t e = launch_q8_quantize_scatter(q, k, v, sb, sh, sn, B, H, N, d, smooth_k, pv_fp8, k_sum, v_amax, rank,
+                                               world, dst, static_cast<uint8_t*>(workspace),
+                                               static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
 dit_status dit_attn_fwd_q8_prequantized(const void* workspace, size_t workspace_bytes, const void* v, void* o, int B,
                                         int H, int N, int d, const int64_t* strides, float scale, int pv_mode,
                                         void* stream) {

@@ -61,6 +61,17 @@ cudaError_t launch_q8_quantize_global(const void* q, const void* k, const void* 
                                       const double* k_sum, const float* v_amax, int64_t n_total, uint8_t* ws,
                                       cudaStream_t stream);
 
+// Fused quantise-and-scatter of a Ulysses group (`world` ranks, this one
+// `rank`): this slice's codes and block scales go straight into the
+// workspaces dst[0..world) of the head-sharded layout (B, H/world heads,
+// world·N tokens), this rank's own V scales into dst[rank]; `ws` holds the
+// slice's statistics.  At most kQ8MaxRanks ranks.
+constexpr int kQ8MaxRanks = 16;
+cudaError_t launch_q8_quantize_scatter(const void* q, const void* k, const void* v, int64_t sb, int64_t sh,
+                                       int64_t sn, int B, int H, int N, int d, int smooth_k, int pv_fp8,
+                                       const double* k_sum, const float* v_amax, int rank, int world,
+                                       uint8_t* const* dst, uint8_t* ws, cudaStream_t stream);
+
 // 8-bit attention over the pre-pass products.  tq8/tk8: 4-D maps over the
 // INT8 codes {d, N, H, B}, box {d, 128, 1, 1} (128-byte swizzle at d = 128,
 // 64-byte at d = 64); tv: e4m3 codes (same box and swizzle, pv_fp8) or the

@@ -21,7 +21,11 @@
 // device reduces its token slice to per-channel K sums and V maxima, the
 // devices combine them (sum, max), and each quantises its own tokens with the
 // combined statistics, so that the 1-byte codes, not the bf16 values, travel
-// in a Ulysses all-to-all.
+// in a Ulysses all-to-all.  launch_q8_quantize_scatter fuses that all-to-all
+// into the quantisers: every code and block scale is stored straight into the
+// workspace of the rank that owns its head in the head-sharded layout (peer
+// memory over NVLink when the ranks are GPUs), so no separate exchange and no
+// local copy of the codes exist.
 //
 // Head dimension d = 128 or 64 (a template argument of every kernel; a
 // thread always covers 8 consecutive channels, one 16-byte load per row).
@@ -65,6 +69,19 @@ __device__ __forceinline__ const uint4* row_ptr(const void* base, int64_t sb, in
                                                 int64_t n) {
     return reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + b * sb + h * sh + n * sn);
 }
+
+// Where a quantiser stores a tensor's codes and block scales.  Without
+// scatter: the slice's own workspace (one entry, hp = H, n_total = N,
+// tok0 = 0).  With scatter: head h of the slice goes to rank h / hp as its
+// head h % hp, its tokens from tok0 on, in a layout of n_total tokens.
+struct Q8Dest {
+    uint8_t* ws[kQ8MaxRanks];
+    int hp;
+    int n_total;
+    int tok0;
+    size_t codes_off;  // byte offset of the codes in a destination workspace
+    size_t scale_off;  // byte offset of the block scales (INT8 tensors)
+};
 
 // grid (n_chunks, B*H).  With G = D/8 channel groups, thread t holds channels
 // [8·(t%G), +8) of rows t/G + (256/G)·i.  Four blocks per SM (64 registers)
@@ -222,7 +239,7 @@ __device__ __forceinline__ uint32_t s8x4(float a, float b, float c, float d) {
 template <int D, int BLK, int THREADS>
 __global__ void __launch_bounds__(THREADS, 1536 / THREADS)
     q8_quant_int8_kernel(const void* __restrict__ x, int64_t sb, int64_t sh, int64_t sn, int H, int N,
-                         const float* __restrict__ mean, int8_t* __restrict__ codes, float* __restrict__ scales) {
+                         const float* __restrict__ mean, const Q8Dest dst) {
     constexpr int kCG = D / 8;
     constexpr int kGroups = THREADS / kCG;  // row groups
     constexpr int kRows = BLK / kGroups;    // rows per thread
@@ -268,7 +285,13 @@ __global__ void __launch_bounds__(THREADS, 1536 / THREADS)
         inv = inv_raw;
         scale = __fdiv_rn(amax, 127.f);
     }
-    if (threadIdx.x == 0) scales[static_cast<int64_t>(bh) * gridDim.x + blockIdx.x] = scale;
+    // destination: rank g, head hh there, rows from tok0 on
+    const int g = h / dst.hp, hh = h - g * dst.hp;
+    const int64_t bh_out = static_cast<int64_t>(b) * dst.hp + hh;
+    int8_t* codes = reinterpret_cast<int8_t*>(dst.ws[g] + dst.codes_off);
+    float* scales = reinterpret_cast<float*>(dst.ws[g] + dst.scale_off);
+    if (threadIdx.x == 0)
+        scales[bh_out * ((dst.n_total + BLK - 1) / BLK) + dst.tok0 / BLK + blockIdx.x] = scale;
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
         const int64_t n = t0 + r0 + kGroups * r;
@@ -280,7 +303,7 @@ __global__ void __launch_bounds__(THREADS, 1536 / THREADS)
             uint2 w;
             w.x = s8x4(q[0], q[1], q[2], q[3]);
             w.y = s8x4(q[4], q[5], q[6], q[7]);
-            *reinterpret_cast<uint2*>(codes + (static_cast<int64_t>(bh) * N + n) * D + cg * 8) = w;
+            *reinterpret_cast<uint2*>(codes + (bh_out * dst.n_total + dst.tok0 + n) * D + cg * 8) = w;
         }
     }
 }
@@ -297,10 +320,13 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 template <int D>
 __global__ void __launch_bounds__(kQuantThreads)
     q8_quant_e4m3_kernel(const void* __restrict__ x, int64_t sb, int64_t sh, int64_t sn, int H, int N,
-                         const float* __restrict__ v_inv, uint8_t* __restrict__ codes) {
+                         const float* __restrict__ v_inv, const Q8Dest dst) {
     constexpr int kCG = D / 8;
     constexpr int kStep = kQuantThreads / kCG;
     const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int g = h / dst.hp, hh = h - g * dst.hp;
+    const int64_t bh_out = static_cast<int64_t>(b) * dst.hp + hh;
+    uint8_t* codes = dst.ws[g] + dst.codes_off;
     const int cg = threadIdx.x % kCG, r0 = threadIdx.x / kCG;
     float inv[8];
 #pragma unroll
@@ -317,7 +343,7 @@ __global__ void __launch_bounds__(kQuantThreads)
                   (e4m3x2(__fmul_rn(f[2], inv[2]), __fmul_rn(f[3], inv[3])) << 16);
             w.y = e4m3x2(__fmul_rn(f[4], inv[4]), __fmul_rn(f[5], inv[5])) |
                   (e4m3x2(__fmul_rn(f[6], inv[6]), __fmul_rn(f[7], inv[7])) << 16);
-            *reinterpret_cast<uint2*>(codes + (static_cast<int64_t>(bh) * N + n) * D + cg * 8) = w;
+            *reinterpret_cast<uint2*>(codes + (bh_out * dst.n_total + dst.tok0 + n) * D + cg * 8) = w;
         }
     }
 }
@@ -341,9 +367,12 @@ __global__ void __launch_bounds__(kFinGroups * D)
 // The K mean and V scales from the combined statistics of all slices
 // (n_total tokens): the arithmetic of q8_finalize_kernel.  D threads.
 template <int D>
+//   With v_scale_own (scatter): this rank (`rank`, heads [rank·hp, +hp) of H)
+//   also stores its heads' V scales into its own destination workspace.
 __global__ void q8_finalize_global_kernel(const double* __restrict__ k_sum, const float* __restrict__ v_amax,
                                           int64_t n_total, int want_sum, int want_vmax, float* __restrict__ k_mean,
-                                          float* __restrict__ v_scale, float* __restrict__ v_inv) {
+                                          float* __restrict__ v_scale, float* __restrict__ v_inv, int H, int hp,
+                                          int rank, float* __restrict__ v_scale_own) {
     const int bh = blockIdx.x, c = threadIdx.x;
     k_mean[bh * D + c] = want_sum ? static_cast<float>(k_sum[bh * D + c] / static_cast<double>(n_total)) : 0.f;
     if (want_vmax) {
@@ -351,6 +380,9 @@ __global__ void q8_finalize_global_kernel(const double* __restrict__ k_sum, cons
         v_scales(v_amax[bh * D + c], sc, inv);
         v_scale[bh * D + c] = sc;
         v_inv[bh * D + c] = inv;
+        const int b = bh / H, h = bh % H;
+        if (v_scale_own != nullptr && h / hp == rank)
+            v_scale_own[(static_cast<int64_t>(b) * hp + (h - rank * hp)) * D + c] = sc;
     }
 }
 
@@ -372,25 +404,48 @@ cudaError_t prepass_d(const void* q, const void* k, const void* v, int64_t sb, i
     return launch_q8_codes(q, k, v, sb, sh, sn, B, H, N, D, smooth_k, pv_fp8, ws, stream);
 }
 
+// The quantisers of Q, K (and V when pv_fp8) for a slice of N tokens whose
+// statistics (K mean, V inverse scales) are in `ws`, storing into `dws`
+// (world workspaces of the layout dL; one entry, the slice's own, without
+// scatter) for heads of hp and tokens from tok0 on.
 template <int D>
-cudaError_t codes_d(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H,
-                    int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
+cudaError_t codes_to(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H,
+                     int N, int smooth_k, int pv_fp8, const uint8_t* ws, uint8_t* const* dws, int world,
+                     const Q8Layout& dL, int hp, int n_total, int tok0, cudaStream_t stream) {
     const Q8Layout L = q8_layout(B, H, N, D, pv_fp8);
     const int BH = B * H;
     const float* k_mean = reinterpret_cast<const float*>(ws + L.k_mean);
     const float* v_inv = reinterpret_cast<const float*>(ws + L.v_inv);
+    Q8Dest dq{};
+    for (int r = 0; r < world; ++r) dq.ws[r] = dws[r];
+    dq.hp = hp;
+    dq.n_total = n_total;
+    dq.tok0 = tok0;
+    Q8Dest dk = dq, dv = dq;
+    dq.codes_off = dL.q_codes;
+    dq.scale_off = dL.q_scale;
+    dk.codes_off = dL.k_codes;
+    dk.scale_off = dL.k_scale;
+    dv.codes_off = dL.v_codes;
+    dv.scale_off = 0;
     // Four rows per thread in both quantisers and at both head sizes.
     constexpr int kQThreads = 4 * D, kKThreads = 2 * D;
     q8_quant_int8_kernel<D, 128, kQThreads><<<dim3((N + 127) / 128, BH), kQThreads, 0, stream>>>(
-        q, sb, sh, sn, H, N, nullptr, reinterpret_cast<int8_t*>(ws + L.q_codes),
-        reinterpret_cast<float*>(ws + L.q_scale));
+        q, sb, sh, sn, H, N, nullptr, dq);
     q8_quant_int8_kernel<D, 64, kKThreads><<<dim3((N + 63) / 64, BH), kKThreads, 0, stream>>>(
-        k, sb, sh, sn, H, N, smooth_k ? k_mean : nullptr, reinterpret_cast<int8_t*>(ws + L.k_codes),
-        reinterpret_cast<float*>(ws + L.k_scale));
+        k, sb, sh, sn, H, N, smooth_k ? k_mean : nullptr, dk);
     if (pv_fp8)
         q8_quant_e4m3_kernel<D><<<dim3((N + 127) / 128, BH), kQuantThreads, 0, stream>>>(v, sb, sh, sn, H, N, v_inv,
-                                                                                         ws + L.v_codes);
+                                                                                         dv);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t codes_d(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B, int H,
+                    int N, int smooth_k, int pv_fp8, uint8_t* ws, cudaStream_t stream) {
+    uint8_t* self[1] = {ws};
+    return codes_to<D>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, self, 1, q8_layout(B, H, N, D, pv_fp8), H,
+                       N, 0, stream);
 }
 
 template <int D>
@@ -416,10 +471,27 @@ cudaError_t quantize_global_d(const void* q, const void* k, const void* v, int64
     q8_finalize_global_kernel<D><<<B * H, D, 0, stream>>>(k_sum, v_amax, n_total, smooth_k, pv_fp8,
                                                           reinterpret_cast<float*>(ws + L.k_mean),
                                                           reinterpret_cast<float*>(ws + L.v_scale),
-                                                          reinterpret_cast<float*>(ws + L.v_inv));
+                                                          reinterpret_cast<float*>(ws + L.v_inv), H, H, 0, nullptr);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_q8_codes(q, k, v, sb, sh, sn, B, H, N, D, smooth_k, pv_fp8, ws, stream);
+}
+
+template <int D>
+cudaError_t quantize_scatter_d(const void* q, const void* k, const void* v, int64_t sb, int64_t sh, int64_t sn, int B,
+                               int H, int N, int smooth_k, int pv_fp8, const double* k_sum, const float* v_amax,
+                               int rank, int world, uint8_t* const* dst, uint8_t* ws, cudaStream_t stream) {
+    const Q8Layout L = q8_layout(B, H, N, D, pv_fp8);
+    const int hp = H / world, n_total = N * world;
+    const Q8Layout dL = q8_layout(B, hp, n_total, D, pv_fp8);
+    q8_finalize_global_kernel<D><<<B * H, D, 0, stream>>>(
+        k_sum, v_amax, n_total, smooth_k, pv_fp8, reinterpret_cast<float*>(ws + L.k_mean),
+        reinterpret_cast<float*>(ws + L.v_scale), reinterpret_cast<float*>(ws + L.v_inv), H, hp, rank,
+        pv_fp8 ? reinterpret_cast<float*>(dst[rank] + dL.v_scale) : nullptr);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return codes_to<D>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, dst, world, dL, hp, n_total, rank * N,
+                       stream);
 }
 
 }  // namespace
@@ -464,6 +536,20 @@ cudaError_t launch_q8_slice_stats(const void* k, const void* v, int64_t sb, int6
                                   cudaStream_t stream) {
     if (d == 128) return slice_stats_d<128>(k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, k_sum, v_amax, stream);
     if (d == 64) return slice_stats_d<64>(k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, ws, k_sum, v_amax, stream);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_q8_quantize_scatter(const void* q, const void* k, const void* v, int64_t sb, int64_t sh,
+                                       int64_t sn, int B, int H, int N, int d, int smooth_k, int pv_fp8,
+                                       const double* k_sum, const float* v_amax, int rank, int world,
+                                       uint8_t* const* dst, uint8_t* ws, cudaStream_t stream) {
+    if (world < 1 || world > kQ8MaxRanks) return cudaErrorInvalidValue;
+    if (d == 128)
+        return quantize_scatter_d<128>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, k_sum, v_amax, rank, world, dst,
+                                       ws, stream);
+    if (d == 64)
+        return quantize_scatter_d<64>(q, k, v, sb, sh, sn, B, H, N, smooth_k, pv_fp8, k_sum, v_amax, rank, world, dst,
+                                      ws, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -8,8 +8,9 @@
  * residual difference that decides whether a denoising step may reuse its
  * cached residual.  Around them: attention over a chunk of the keys with its
  * log-sum-exp and the merge of chunks, the 8-bit pre-pass split for a
- * token-sharded sequence, the error of one output against another, and (in
- * dit_cache.h) step-cache policies whose decisions stay on the device.
+ * token-sharded sequence (with a fused quantise-and-scatter for the Ulysses
+ * all-to-all), the error of one output against another, and (in dit_cache.h)
+ * step-cache policies whose decisions stay on the device.
  *
  * Conventions shared by every entry point
  *   - Every buffer is caller-owned device memory.  The library allocates no
@@ -208,6 +209,41 @@ dit_status dit_attn_q8_quantize_global(const void* q, const void* k, const void*
 dit_status dit_attn_fwd_q8_prequantized(const void* workspace, size_t workspace_bytes, const void* v, void* o,
                                         int B, int H, int N, int d, const int64_t* strides, float scale,
                                         int pv_mode, void* stream);
+
+/*
+ * dit_attn_q8_quantize_scatter — steps 2 and 3 above in one launch sequence:
+ * the quantisers of dit_attn_q8_quantize_global store every code and block
+ * scale of this rank's slice straight into the workspace of the rank that
+ * owns its head after the all-to-all, so no separate exchange of the codes
+ * runs.  Same sources: ParaAttention, "Context Parallelism"; the TMAP
+ * image-to-video blog's sequence parallelism with 8-bit attention.
+ *
+ *   q, k, v, B, H, N, d, strides, smooth_k, pv_mode, k_sum, v_amax
+ *                  as dit_attn_q8_quantize_global, for this rank's slice of N
+ *                  tokens (the combined statistics of all world·N tokens).
+ *   rank, world    this rank and the group size, 1 <= world <= 16; H must be
+ *                  a multiple of world and, when world > 1, N of 128.
+ *   dst_workspaces host array of `world` device pointers: the workspace of
+ *                  each rank for the head-sharded problem (B, H/world heads,
+ *                  world·N tokens), dit_attn_q8_workspace_bytes of it, 256-byte
+ *                  aligned, pairwise disjoint.  Entry r receives this slice's
+ *                  codes and scales of heads [r·H/world, (r+1)·H/world) at
+ *                  token offset rank·N; entry `rank` also receives this rank's
+ *                  heads' V scales (FP8 mode).  On a multi-GPU node the other
+ *                  entries are peer-mapped device memory (P2P stores over
+ *                  NVLink); the caller makes every rank's stores complete
+ *                  (stream synchronisation and a group barrier) before any
+ *                  rank runs dit_attn_fwd_q8_prequantized on its entry.
+ *   workspace      this rank's slice workspace (dit_attn_q8_workspace_bytes for
+ *                  B, H, N): receives the K mean and V scales.
+ * Errors as dit_attn_q8_quantize_global; DIT_ERR_WORKSPACE for a destination
+ * that is too small, misaligned or overlapping another buffer.
+ */
+dit_status dit_attn_q8_quantize_scatter(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                                        const int64_t* strides, int smooth_k, int pv_mode, const double* k_sum,
+                                        const float* v_amax, int rank, int world, void* const* dst_workspaces,
+                                        size_t dst_workspace_bytes, void* workspace, size_t workspace_bytes,
+                                        void* stream);
 
 /*
  * fbc_rel_l1 — first-block-cache residual difference and decision:

@@ -312,5 +312,29 @@ def test_sharded_q8_argument_errors(lib):
     assert pq(ws=WS + 128) == dit.DIT_ERR_WORKSPACE
 
 
+def test_quantize_scatter_argument_errors(lib):
+    # all rejected on the host before any launch (the pointers are never touched)
+    wsb = lib.dit_attn_q8_workspace_bytes(1, 4, 256, 128, 0)
+    dwb = lib.dit_attn_q8_workspace_bytes(1, 2, 512, 128, 0)
+    KS, VA = 0x62000000, 0x63000000
+    D0, D1 = 0x64000000, 0x64000000 + ((dwb + 255) // 256) * 256
+
+    def sc(world=2, rank=0, H=4, N=256, dst=(D0, D1), dwb=dwb, ks=KS):
+        arr = (ctypes.c_void_p * len(dst))(*dst) if dst is not None else None
+        return lib.dit_attn_q8_quantize_scatter(Q, K, V, 1, H, N, 128, None, 1, 0, ks, VA, rank, world, arr, dwb,
+                                                WS, wsb, None)
+    assert sc(world=0, dst=()) == dit.DIT_ERR_INVALID_ARG
+    assert sc(world=17, dst=(D0,) * 17) == dit.DIT_ERR_INVALID_ARG
+    assert sc(rank=2) == dit.DIT_ERR_INVALID_ARG
+    assert sc(H=3) == dit.DIT_ERR_INVALID_ARG                      # heads do not split over the ranks
+    assert sc(N=200) == dit.DIT_ERR_INVALID_ARG                    # whole 128-token blocks per rank
+    assert sc(dst=None) == dit.DIT_ERR_INVALID_ARG
+    assert sc(ks=0) == dit.DIT_ERR_INVALID_ARG
+    assert sc(dwb=dwb - 256) == dit.DIT_ERR_WORKSPACE
+    assert sc(dst=(D0, D0 + 256)) == dit.DIT_ERR_WORKSPACE         # destinations overlap
+    assert sc(dst=(D0, D1 + 128)) == dit.DIT_ERR_WORKSPACE         # not 256-byte aligned
+    assert sc(dst=(D0, WS)) == dit.DIT_ERR_WORKSPACE               # the slice workspace itself
+
+
 def test_wait_selftest_argument_error(lib):
     assert lib.dit_wait_selftest(None, None) == dit.DIT_ERR_INVALID_ARG

@@ -13,7 +13,9 @@ ranks meeting at a host barrier.  No kernel waits on another rank's kernel.
 The gathered outputs must match the oracle's full-sequence results, and the
 Ulysses outputs must equal the single-device calls bit for bit (every head
 sees the same keys in the same order).  A layout slip between the all-to-all
-and the kernels' strides fails here.
+and the kernels' strides fails here.  The 8-bit Ulysses runs both with the
+code all-to-all and with the fused quantise-and-scatter, each rank's
+quantisers storing into every rank's workspace (here all on the one GPU).
 """
 import threading
 
@@ -88,6 +90,17 @@ class LocalComm:
         self._done()
         return []
 
+    def shared_workspace(self, nbytes, device):
+        buf = torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+        parts = self._gather(buf)
+        ptrs = [t.data_ptr() for t in parts]
+        self._done()
+        return buf, ptrs
+
+    def barrier(self):
+        torch.cuda.synchronize()
+        self.hub.barrier.wait()
+
 
 def _run_ranks(world, fn):
     """fn(rank, comm) on `world` threads; returns the per-rank results."""
@@ -132,9 +145,10 @@ def test_ulysses_with_the_kernels(world, d):
     assert_bf16_parity(from_device_bf16(o[:, :, rows]), oracle.attention(q, k, v, rows=rows), f"ulysses P={world}")
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["all-to-all", "scatter"])
 @pytest.mark.parametrize("world", [2, 4])
 @pytest.mark.parametrize("pv_mode", ["fp8", "bf16"])
-def test_ulysses_q8_with_the_kernels(world, pv_mode):
+def test_ulysses_q8_with_the_kernels(world, pv_mode, fused):
     import diffusion_transformer_attention_attn_b200 as dit
     from diffusion_transformer_attention_attn_b200 import context_parallel as cp
     (q, k, v), (qd, kd, vd) = _case(8, 1024, 128, seed=50 + world, k_offset_std=3.0, zero_q_channel=7)
@@ -142,7 +156,7 @@ def test_ulysses_q8_with_the_kernels(world, pv_mode):
     sl = [slice(r * Nl, (r + 1) * Nl) for r in range(world)]
     outs = _run_ranks(world, lambda r, comm: cp.ulysses_attention_q8(
         qd[:, :, sl[r]].contiguous(), kd[:, :, sl[r]].contiguous(), vd[:, :, sl[r]].contiguous(), smooth_k=True,
-        pv_mode=pv_mode, comm=comm))
+        pv_mode=pv_mode, comm=comm, fused=fused))
     o = torch.cat(outs, dim=2)
     assert torch.equal(o, dit.dit_attn_fwd_q8(qd, kd, vd, smooth_k=True, pv_mode=pv_mode))
     rows = np.arange(0, 1024, 7)

@@ -129,6 +129,58 @@ def test_split_entry_points_match_the_oracle(d, pv_mode, smooth_k):
     assert c >= 0.9995 and r <= (3.5e-2 if fp8 else 5e-3), (c, r)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("pv_mode", ["fp8", "bf16"])
+@pytest.mark.parametrize("world", [2, 4])
+def test_quantize_scatter_matches_the_oracle_and_the_single_call(world, pv_mode, d):
+    # Each rank's quantisers store straight into every rank's head-sharded
+    # workspace (the fused all-to-all).  The ranks run one after another on the
+    # one GPU; each writes disjoint parts of the destinations.
+    dit = _dit()
+    H, N = 8, 1024
+    case = inputs.AttnCase(f"scat{d}", 1, H, N, d, k_offset_std=3.0, zero_q_channel=5, seed=17)
+    q, k, v = inputs.attn_inputs(case)
+    qd, kd, vd = (to_device_bf16(t) for t in (q, k, v))
+    B, fp8 = 1, pv_mode == "fp8"
+    Nl, hp = N // world, H // world
+    sl = [slice(r * Nl, (r + 1) * Nl) for r in range(world)]
+    stats = [dit.dit_attn_q8_channel_stats(kd[:, :, s], vd[:, :, s], smooth_k=True, pv_mode=pv_mode) for s in sl]
+    k_sum = sum(x for x, _ in stats)
+    v_amax = torch.stack([y for _, y in stats]).amax(dim=0)
+    nbytes = dit.dit_attn_q8_workspace_bytes(B, hp, N, d, pv_mode)
+    dst = [torch.full((nbytes,), 0x5A, dtype=torch.uint8, device="cuda") for _ in range(world)]
+    ptrs = [t.data_ptr() for t in dst]
+    for r, s in enumerate(sl):
+        dit.dit_attn_q8_quantize_scatter(qd[:, :, s].contiguous(), kd[:, :, s].contiguous(),
+                                         vd[:, :, s].contiguous(), k_sum, v_amax, r, world, ptrs, nbytes,
+                                         smooth_k=True, pv_mode=pv_mode)
+    torch.cuda.synchronize()
+    # codes and scales of every destination against the oracle's whole-sequence quantisers
+    mean = oracle.mean_from_sums(oracle.k_channel_sums(k), N)
+    qc, qs = oracle.quant_int8_blocks(q, 128)
+    kc, ks = oracle.quant_int8_blocks(k, 64, mean)
+    vc, vs = oracle.quant_e4m3_with_amax(v, oracle.channel_amax(v))
+    out = torch.empty_like(qd)
+    for g in range(world):
+        heads = slice(g * hp, (g + 1) * hp)
+        got = {n: t.cpu().numpy() for n, t in dit.q8_views(dst[g], B, hp, N, d, pv_mode).items()}
+        np.testing.assert_array_equal(got["q_codes"], qc[:, heads])
+        np.testing.assert_array_equal(got["q_scale"], qs[:, heads])
+        np.testing.assert_array_equal(got["k_codes"], kc[:, heads])
+        np.testing.assert_array_equal(got["k_scale"], ks[:, heads])
+        if fp8:
+            np.testing.assert_array_equal(got["v_codes"], vc[:, heads])
+            np.testing.assert_array_equal(got["v_scale"], vs[:, heads])
+        vh = None if fp8 else vd[:, heads].contiguous()
+        out[:, heads] = dit.dit_attn_fwd_q8_prequantized(dst[g], B, hp, N, v=vh, pv_mode=pv_mode, d=d)
+    torch.cuda.synchronize()
+    assert torch.equal(out, dit.dit_attn_fwd_q8(qd, kd, vd, smooth_k=True, pv_mode=pv_mode))
+    o = from_device_bf16(out)
+    ref = oracle.attention(q, k, v)
+    c, r = cosine(o, ref), rel_l1(o, ref)
+    assert c >= Q8_COSINE and r <= (FP8_REL_L1 if fp8 else Q8_REL_L1), (c, r)
+
+
 @pytest.mark.parametrize("pv_mode", ["fp8", "bf16"])
 @pytest.mark.parametrize("smooth_k", [True, False])
 @pytest.mark.parametrize("world", [2, 4])
