@@ -148,7 +148,8 @@ def test_deterministic():
 
 # ---------------------------------------------------------------- full-size workloads, sampled rows
 
-@pytest.mark.parametrize("case,count", [(inputs.IMAGE, 96), (inputs.VIDEO_MID, 24), (inputs.VIDEO_LONG, 64)],
+@pytest.mark.parametrize("case,count", [(inputs.IMAGE, 96), (inputs.VIDEO_MID, 24), (inputs.VIDEO_LONG, 64),
+                                        (inputs.AttnCase("image_b1h24n4608d64", 1, 24, 4608, 64, seed=27), 96)],
                          ids=lambda x: getattr(x, "name", str(x)))
 def test_full_size_sampled_rows(case, count):
     import diffusion_transformer_attention_attn_b200 as dit
