@@ -248,6 +248,14 @@ __global__ void __launch_bounds__(THREADS, 1536 / THREADS)
     const int bh = blockIdx.y, b = bh / H, h = bh % H;
     const int cg = threadIdx.x % kCG, r0 = threadIdx.x / kCG;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * BLK;
+    // destination: rank g, head hh there, rows from tok0 on (worked out
+    // before the loads, off the path between the block reduction and the stores)
+    const int g = h / dst.hp, hh = h - g * dst.hp;
+    const int64_t bh_out = static_cast<int64_t>(b) * dst.hp + hh;
+    int8_t* const codes = reinterpret_cast<int8_t*>(dst.ws[g] + dst.codes_off) +
+                          (bh_out * dst.n_total + dst.tok0) * D + cg * 8;
+    float* const scale_out = reinterpret_cast<float*>(dst.ws[g] + dst.scale_off) +
+                             bh_out * ((dst.n_total + BLK - 1) / BLK) + dst.tok0 / BLK + blockIdx.x;
     float mu[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) mu[i] = mean ? mean[bh * D + cg * 8 + i] : 0.f;
@@ -285,13 +293,7 @@ __global__ void __launch_bounds__(THREADS, 1536 / THREADS)
         inv = inv_raw;
         scale = __fdiv_rn(amax, 127.f);
     }
-    // destination: rank g, head hh there, rows from tok0 on
-    const int g = h / dst.hp, hh = h - g * dst.hp;
-    const int64_t bh_out = static_cast<int64_t>(b) * dst.hp + hh;
-    int8_t* codes = reinterpret_cast<int8_t*>(dst.ws[g] + dst.codes_off);
-    float* scales = reinterpret_cast<float*>(dst.ws[g] + dst.scale_off);
-    if (threadIdx.x == 0)
-        scales[bh_out * ((dst.n_total + BLK - 1) / BLK) + dst.tok0 / BLK + blockIdx.x] = scale;
+    if (threadIdx.x == 0) *scale_out = scale;
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
         const int64_t n = t0 + r0 + kGroups * r;
@@ -303,7 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1536 / THREADS)
             uint2 w;
             w.x = s8x4(q[0], q[1], q[2], q[3]);
             w.y = s8x4(q[4], q[5], q[6], q[7]);
-            *reinterpret_cast<uint2*>(codes + (bh_out * dst.n_total + dst.tok0 + n) * D + cg * 8) = w;
+            *reinterpret_cast<uint2*>(codes + n * D) = w;
         }
     }
 }
@@ -326,8 +328,8 @@ __global__ void __launch_bounds__(kQuantThreads)
     const int bh = blockIdx.y, b = bh / H, h = bh % H;
     const int g = h / dst.hp, hh = h - g * dst.hp;
     const int64_t bh_out = static_cast<int64_t>(b) * dst.hp + hh;
-    uint8_t* codes = dst.ws[g] + dst.codes_off;
     const int cg = threadIdx.x % kCG, r0 = threadIdx.x / kCG;
+    uint8_t* const codes = dst.ws[g] + dst.codes_off + (bh_out * dst.n_total + dst.tok0) * D + cg * 8;
     float inv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) inv[i] = v_inv[bh * D + cg * 8 + i];
@@ -343,7 +345,7 @@ __global__ void __launch_bounds__(kQuantThreads)
                   (e4m3x2(__fmul_rn(f[2], inv[2]), __fmul_rn(f[3], inv[3])) << 16);
             w.y = e4m3x2(__fmul_rn(f[4], inv[4]), __fmul_rn(f[5], inv[5])) |
                   (e4m3x2(__fmul_rn(f[6], inv[6]), __fmul_rn(f[7], inv[7])) << 16);
-            *reinterpret_cast<uint2*>(codes + (bh_out * dst.n_total + dst.tok0 + n) * D + cg * 8) = w;
+            *reinterpret_cast<uint2*>(codes + n * D) = w;
         }
     }
 }
