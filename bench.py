@@ -21,6 +21,8 @@ Under torchrun (N > 1) every rank runs its own replica of the workload (weak
 scaling; no data-path collective), timed as the max over ranks.
 `--impl reference` times the fp64 CPU oracle on a bounded sample of the same
 workload on the host cores (rank 0 only).
+At N=1 the line also carries `library_context`: cuDNN's fused attention
+(torch SDPA, cuDNN backend) timed on the same bf16 inputs, for comparison only.
 """
 from __future__ import annotations
 
@@ -242,6 +244,31 @@ def _time_calls(torch, stream, fn, reps):
     ev[1].record(stream)
     ev[1].synchronize()
     return ev[0].elapsed_time(ev[1]) / reps
+
+
+def library_context(torch, dev, stream, dq, dk, dv, do, attn_ms, flops, reps):
+    """NVIDIA's own fused attention on the same bf16 inputs, for context only.
+
+    torch's scaled_dot_product_attention restricted to its cuDNN backend
+    (cuDNN's sm100 flash forward kernel), timed like this library's call with
+    CUDA events on the same stream, after one untimed call whose output is
+    compared with this library's.  Nothing of this library's path uses it.
+    """
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        sdpa = torch.nn.functional.scaled_dot_product_attention
+        with torch.cuda.stream(stream), sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            out = sdpa(dq, dk, dv)
+            torch.cuda.synchronize(dev)
+            cos = torch.nn.functional.cosine_similarity(out.float().flatten(), do.float().flatten(), dim=0).item()
+            del out
+            lib_ms = _time_calls(torch, stream, lambda: sdpa(dq, dk, dv), reps)
+    except Exception as e:  # a box without cuDNN's fused attention: report, do not fail the bench
+        return {"cudnn_sdpa_bf16": f"unavailable: {e!r}"[:200]}
+    return {"what": "torch SDPA, cuDNN backend only (cuDNN's sm100 flash forward), same bf16 inputs and stream",
+            "cudnn_sdpa_bf16_ms": lib_ms, "cudnn_sdpa_bf16_tflops": flops / (lib_ms * 1e-3) / 1e12,
+            "this_library_bf16_ms": attn_ms, "this_library_over_cudnn_time_ratio": attn_ms / lib_ms,
+            "cosine_vs_this_library": cos}
 
 
 CHUNKS = 4  # key chunks of the one-GPU ring emulation
@@ -650,6 +677,8 @@ def run_ours(args):
         line["roofline"], line["roofline_other"] = roof_bf16, roof_q8
     else:
         line["roofline"], line["roofline_other"] = roof_q8, roof_bf16
+    if ws == 1 and rank == 0 and not args.no_library_context:
+        line["library_context"] = library_context(torch, dev, stream, dq, dk, dv, do, attn_ms, flops, max(2, min(K, 5)))
     if ws == 1 and rank == 0 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
@@ -681,6 +710,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="video_long",
                     help="video_long is the benchmark; the others serve profiling captures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-library-context", action="store_true",
+                    help="skip the cuDNN fused-attention timing reported beside this library's")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the step-cache, comparison, merge and chunked-attention timings")
     args = ap.parse_args(argv)
