@@ -251,6 +251,47 @@ def test_fp8_kernel_tracks_quantised_emulation():
     assert cosine(out, emu) >= 0.9995 and rel_l1(out, emu) <= 3.5e-2
 
 
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("mode", ["fp8", "bf16"])
+def test_growing_logits_rescaling_path(mode, d):
+    # Logits grow along the key axis, so each row's running max moves past the
+    # rescale threshold tile after tile (2 in log2 units with FP8 P, 8 with bf16
+    # P) and O is rescaled in tensor memory again and again.  Logits this large
+    # magnify the INT8 rounding of Q and K beyond the 8-bit bar, so the kernel
+    # is held to the fp64 attention over the same dequantised codes (which
+    # models everything but P's own rounding), and to the exact attention only
+    # loosely.  V is scaled by 1/4 so the nearly one-hot rows keep |O| in the
+    # workloads' range.
+    case = inputs.AttnCase("q8grow", 1, 2, 1024, d, seed=71)
+    q, k, v = inputs.attn_inputs(case)
+    qf = inputs.bf16_to_f32(q) * np.float32(3.0)
+    ramp = np.linspace(0.0, 4.0, case.N, dtype=np.float32)[None, None, :, None]
+    kf = inputs.bf16_to_f32(k) * (1.0 + ramp)
+    q, k = inputs.bf16_bits(qf), inputs.bf16_bits(kf)
+    v = inputs.bf16_bits(inputs.bf16_to_f32(v) * np.float32(0.25))
+    out = _run(q, k, v, mode)
+    assert np.isfinite(out).all()
+    if mode == "fp8":
+        emu = oracle.emulated_q8_attention(q, k, v, smooth_k=True)
+    else:
+        # bf16 P·V keeps V in bf16: only Q and K are dequantised codes
+        qc, qs = oracle.quant_int8_blocks(q, 128)
+        kc, ks = oracle.quant_int8_blocks(k, 64, oracle.channel_mean(k))
+        tok = np.arange(case.N)
+        qd = qc.astype(np.float64) * qs[:, :, tok // 128, None].astype(np.float64)
+        kd = kc.astype(np.float64) * ks[:, :, tok // 64, None].astype(np.float64)
+        emu = oracle.attention(qd, kd, inputs.bf16_to_f32(v).astype(np.float64))
+    c, r = cosine(out, emu), rel_l1(out, emu)
+    print(f"growing logits d={d} [{mode}] vs dequantised fp64: cos={c:.6f} relL1={r:.3e}")
+    if mode == "fp8":
+        assert c >= 0.9995 and r <= 3.5e-2, (c, r)
+    else:
+        assert c >= 0.99999 and r <= 5e-3, (c, r)
+    ref = oracle.attention(q, k, v)
+    print(f"  vs exact fp64: cos={cosine(out, ref):.6f} relL1={rel_l1(out, ref):.3e}")
+    assert cosine(out, ref) >= 0.995
+
+
 def test_smoothing_is_softmax_invariant():
     # Adding a per-channel offset to every key leaves the smoothed path's
     # quantised K unchanged up to rounding: outputs agree closely.
