@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < nkv; ++j) {
             const int s = j % C::kStages;
             const uint32_t ph = (j / C::kStages) & 1;
-            if (j >= C::kStages && !mbar_wait(&bars.k_empty[s], ph ^ 1, abort_flag, err)) break;
+            if (j >= C::kStages && !mbar_wait_lean(&bars.k_empty[s], ph ^ 1, abort_flag, err)) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars.k_full[s], C::kTileBytes);
                 for (int hf = 0; hf < C::kHalves; ++hf)
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             ++nk[s];
-            if (j >= C::kStages && !mbar_wait(&bars.v_empty[s], ph ^ 1, abort_flag, err)) break;
+            if (j >= C::kStages && !mbar_wait_lean(&bars.v_empty[s], ph ^ 1, abort_flag, err)) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars.v_full[s], C::kTileBytes);
                 for (int hf = 0; hf < C::kHalves; ++hf)
@@ -240,7 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < D / 16; ++kk)
                 mma_ss<0>(tS, sdesc_add(dQ, kmajor_off(kk)), sdesc_add(dK, kmajor_off(kk)), C::kIdescQK, kk > 0);
         };
-        bool ok = mbar_wait(bars.q_full, 0, abort_flag, err) && mbar_wait(&bars.k_full[0], 0, abort_flag, err);
+        bool ok = mbar_wait_lean(bars.q_full, 0, abort_flag, err) &&
+                  mbar_wait_lean(&bars.k_full[0], 0, abort_flag, err);
         if (ok) {
             tc_fence_after();
             issue_s(tS0, dQ0, dK0);
@@ -255,14 +256,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool more = j + 1 < nkv;
                 const int ks = (j + 1) % C::kStages;
                 const SDesc dK = sdesc_add(dK0, ks * C::kTileBytes);
-                ok = mbar_wait(&bars.v_full[vs], (j / C::kStages) & 1, abort_flag, err);
+                ok = mbar_wait_lean(&bars.v_full[vs], (j / C::kStages) & 1, abort_flag, err);
                 if (!ok) break;
                 // O_t += P_t·V (in two 64-key halves when P is published in halves).
                 auto issue_pv = [&](int t, uint32_t tO, uint32_t tP) {
                     constexpr int kParts = kSplitP ? 2 : 1;
 #pragma unroll
                     for (int hf = 0; hf < kParts; ++hf) {
-                        ok = ok && mbar_wait(&bars.p_full[2 * t + hf], j & 1, abort_flag, err);
+                        ok = ok && mbar_wait_lean(&bars.p_full[2 * t + hf], j & 1, abort_flag, err);
                         if (!ok) return;
                         tc_fence_after();
 #pragma unroll
@@ -276,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(&bars.o_ready[0]);
                 __syncwarp();
                 if (more) {
-                    ok = mbar_wait(&bars.k_full[ks], ((j + 1) / C::kStages) & 1, abort_flag, err);
+                    ok = mbar_wait_lean(&bars.k_full[ks], ((j + 1) / C::kStages) & 1, abort_flag, err);
                     if (!ok) break;
                     tc_fence_after();
                     issue_s(tS0, dQ0, dK);
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float l = 0.f;
         bool ok = true;
         for (int j = 0; j < nkv; ++j) {
-            ok = mbar_wait(&bars.s_full[wg], j & 1, abort_flag, err);
+            ok = mbar_wait_lean(&bars.s_full[wg], j & 1, abort_flag, err);
             if (!ok) break;
             tc_fence_after();
             uint32_t r[kBN / 32][32];
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool need = m_new > m + 8.0f;
                 if (__any_sync(0xffffffffu, need)) {
                     // O holds P_{<j}·V; rescale it once P_{j-1}·V has landed.
-                    ok = mbar_wait(&bars.o_ready[wg], (j - 1) & 1, abort_flag, err);
+                    ok = mbar_wait_lean(&bars.o_ready[wg], (j - 1) & 1, abort_flag, err);
                     if (!ok) break;
                     tc_fence_after();
                     const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
@@ -435,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             l += lsum.x + lsum.y;
         }
         // Epilogue: O / l -> bf16 -> global (rows at or past Nq are padding).
-        if (ok) ok = mbar_wait(&bars.o_ready[wg], (nkv - 1) & 1, abort_flag, err);
+        if (ok) ok = mbar_wait_lean(&bars.o_ready[wg], (nkv - 1) & 1, abort_flag, err);
         if (ok) {
             tc_fence_after();
             const float inv_l = 1.0f / l;

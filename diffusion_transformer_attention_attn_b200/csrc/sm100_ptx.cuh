@@ -75,6 +75,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
+// The same wait, polling 16 times between the checks of the abort word and
+// the clock instead of keeping a poll counter: fewer instructions per poll on
+// the SMSPs the waiting warps share with busy ones.  The bf16 attention kernel
+// measured 2% faster with it; the 8-bit kernel measured 2% slower, so it keeps
+// mbar_wait.
+__device__ __forceinline__ bool mbar_wait_lean(uint64_t* bar, uint32_t parity, volatile int* abort, int* err) {
+    bool ok = mbar_try_wait(bar, parity);
+    if (!ok) {
+        const uint64_t t0 = globaltimer();
+        for (;;) {
+            bool got = false;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                if (mbar_try_wait(bar, parity)) {
+                    got = true;
+                    break;
+                }
+            }
+            if (got) {
+                ok = true;
+                break;
+            }
+            if (*abort) break;
+            if (globaltimer() - t0 > kWaitLimitNs) {
+                *abort = 1;
+                atomicExch(err, kErrTimeout);
+                break;
+            }
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
 // Drain wait used on the way out of an aborted kernel: ignores the abort word
 // (the copy or MMA being waited for still lands) but stays bounded in time.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
