@@ -51,7 +51,7 @@ SPEC_BF16_TFLOPS = 2250.0
 # ncu capture on the 45760-token, 24-head video workload, scaled by N:
 # each head's K/V stays L2-resident while its CTAs run, so traffic grows with N.
 # Set to None whenever the kernel changes until it is captured again.
-BF16_ATTN_DRAM_BYTES_AT = (1.122631e9, 45760)
+BF16_ATTN_DRAM_BYTES_AT = (1.1227456e9, 45760)
 SPEC_HBM_GBS = 8000.0
 
 
